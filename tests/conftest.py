@@ -1,0 +1,20 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a) and the built library")
+    config.addinivalue_line("markers", "slow: full-size parity case (minutes)")
+
+
+@pytest.fixture(scope="session")
+def page_facts():
+    import json
+    with open(os.path.join(ROOT, "tests", "golden", "page_facts.json")) as f:
+        return json.load(f)
