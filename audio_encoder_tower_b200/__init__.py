@@ -1,0 +1,8 @@
+"""B200-native (sm_100a) Whisper-style audio encoder tower.
+
+The compute lives in libenc_b200.so (hand-written CUDA behind the C ABI of
+include/enc.h); this package only builds it and binds it with ctypes.
+"""
+from .binding import Encoder, EncError, load_library, status_string  # noqa: F401
+
+__all__ = ["Encoder", "EncError", "load_library", "status_string"]

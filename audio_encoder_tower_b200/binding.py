@@ -1,0 +1,213 @@
+"""ctypes binding of the encoder C ABI (include/enc.h).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of libenc_b200.so. PyTorch provides device memory and streams.
+The library must be built (python -m audio_encoder_tower_b200.build); there is
+no fallback of any kind when it is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libenc_b200.so")
+
+ENC_OK, ENC_ERR_INVALID_ARG, ENC_ERR_UNSUPPORTED, ENC_ERR_OOM, ENC_ERR_CUDA, ENC_ERR_TIMEOUT, \
+    ENC_ERR_DEVICE_CHECK = range(7)
+ENC_DTYPE_BF16, ENC_DTYPE_FP32 = 0, 1
+
+EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status", "enc_destroy",
+            "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16"]
+
+
+class EncError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+class EncConfig(ctypes.Structure):
+    _fields_ = [("n_mels", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ffn_dim", ctypes.c_int32),
+                ("max_frames", ctypes.c_int32), ("max_batch", ctypes.c_int32), ("pool_step", ctypes.c_int32),
+                ("proj_hidden", ctypes.c_int32), ("proj_out", ctypes.c_int32), ("ln_eps", ctypes.c_float),
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+_VP = ctypes.c_void_p
+_VPP = ctypes.POINTER(ctypes.c_void_p)
+LAYER_FIELDS = ["ln1_g", "ln1_b", "q_w", "q_b", "k_w", "k_b", "v_w", "v_b", "o_w", "o_b", "ln2_g", "ln2_b",
+                "fc1_w", "fc1_b", "fc2_w", "fc2_b"]
+
+
+class EncWeights(ctypes.Structure):
+    _fields_ = ([("conv1_w", _VP), ("conv1_b", _VP), ("conv2_w", _VP), ("conv2_b", _VP)] +
+                [(f, _VPP) for f in LAYER_FIELDS] +
+                [("lnpost_g", _VP), ("lnpost_b", _VP), ("proj1_w", _VP), ("proj1_b", _VP),
+                 ("proj2_w", _VP), ("proj2_b", _VP)])
+
+
+_LIB = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libenc_b200.so and declare the signatures of every exported call."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m audio_encoder_tower_b200.build`")
+    lib = ctypes.CDLL(path)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.enc_create.argtypes = [ctypes.POINTER(EncConfig), ctypes.POINTER(EncWeights), ctypes.POINTER(ctypes.c_void_p)]
+    lib.enc_create.restype = ctypes.c_int
+    lib.enc_forward.argtypes = [_VP, _VP, i32p, ctypes.c_int32, _VP, _VP]
+    lib.enc_forward.restype = ctypes.c_int
+    lib.enc_output_positions.argtypes = [_VP, ctypes.c_int32, i32p, i32p, i32p, i32p]
+    lib.enc_output_positions.restype = ctypes.c_int
+    lib.enc_get_status.argtypes = [_VP, _VP]
+    lib.enc_get_status.restype = ctypes.c_int
+    lib.enc_destroy.argtypes = [_VP]
+    lib.enc_destroy.restype = None
+    lib.enc_status_string.argtypes = [ctypes.c_int]
+    lib.enc_status_string.restype = ctypes.c_char_p
+    lib.enc_device_bytes.argtypes = [_VP]
+    lib.enc_device_bytes.restype = ctypes.c_size_t
+    lib.enc_linear_bf16.argtypes = [_VP, _VP, _VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                    ctypes.c_int32, _VP, _VP]
+    lib.enc_linear_bf16.restype = ctypes.c_int
+    lib.enc_attention_bf16.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP]
+    lib.enc_attention_bf16.restype = ctypes.c_int
+    _LIB = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().enc_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != ENC_OK:
+        raise EncError(code, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Encoder:
+    """One encoder handle (enc_create / enc_forward / enc_destroy).
+
+    weights: dict of device tensors in PyTorch layouts named as in enc.h
+    ("conv1_w", "layers.{l}.q_w", "lnpost_g", "proj1_w", ...), dtype matching
+    `dtype` ("bf16" or "fp32"). They may be freed after construction.
+    """
+
+    def __init__(self, *, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
+                 pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, weights: dict):
+        self.lib = load_library()
+        self.cfg = EncConfig(n_mels, d_model, n_layers, n_heads, head_dim, ffn_dim, max_frames, max_batch,
+                             pool_step, proj_hidden, proj_out, ln_eps,
+                             ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0)
+        w = EncWeights()
+        for f in ("conv1_w", "conv1_b", "conv2_w", "conv2_b", "lnpost_g", "lnpost_b",
+                  "proj1_w", "proj1_b", "proj2_w", "proj2_b"):
+            setattr(w, f, _ptr(weights.get(f)))
+        keep = []
+        for f in LAYER_FIELDS:
+            arr = (ctypes.c_void_p * max(n_layers, 1))()
+            for l in range(n_layers):
+                arr[l] = _ptr(weights.get(f"layers.{l}.{f}"))
+            keep.append(arr)
+            setattr(w, f, ctypes.cast(arr, _VPP))
+        h = ctypes.c_void_p()
+        _check(self.lib.enc_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h)), "enc_create")
+        self.handle = h
+        self.dtype = dtype
+
+    # ----------------------------------------------------------- geometry
+    def output_positions(self, B: int, lengths=None):
+        """(n_out [B] int32, p_out, d_out) for a batch, from the library."""
+        n_out = np.zeros(B, np.int32)
+        p = ctypes.c_int32()
+        dd = ctypes.c_int32()
+        lp = None
+        if lengths is not None:
+            lengths = np.ascontiguousarray(lengths, dtype=np.int32)
+            lp = lengths.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        _check(self.lib.enc_output_positions(self.handle, B, lp, n_out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                             ctypes.byref(p), ctypes.byref(dd)), "enc_output_positions")
+        return n_out, p.value, dd.value
+
+    # ------------------------------------------------------------ forward
+    def forward(self, mel, lengths=None, out=None, stream=None):
+        """Enqueue the forward pass of mel [B, n_mels, T] (device) on `stream`.
+
+        Returns `out` [B, P_out, d_out] (allocated with torch when not given).
+        """
+        import torch
+        B = int(mel.shape[0])
+        if out is None:
+            _, p_out, d_out = self.output_positions(B, lengths)
+            out = torch.empty((B, p_out, d_out), dtype=mel.dtype, device=mel.device)
+        lp = None
+        if lengths is not None:
+            self._len = np.ascontiguousarray(lengths, dtype=np.int32)
+            lp = self._len.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        _check(self.lib.enc_forward(self.handle, _ptr(mel), lp, B, _ptr(out), _stream_handle(stream)),
+               "enc_forward")
+        return out
+
+    def status(self, stream=None):
+        """Synchronise `stream` and raise if a device-side check or wait failed."""
+        _check(self.lib.enc_get_status(self.handle, _stream_handle(stream)), "enc_get_status")
+
+    def device_bytes(self) -> int:
+        return int(self.lib.enc_device_bytes(self.handle))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.enc_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ------------------------------------------------------- single-kernel calls
+def linear_bf16(A, W, bias=None, out=None, resid=None, gelu=False, status=None, stream=None):
+    """out = act(A W^T + bias) on the tensor cores (bf16 in/out), or resid += A W^T + bias."""
+    import torch
+    M, K = A.shape
+    N = W.shape[0]
+    if out is None and resid is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check(load_library().enc_linear_bf16(_ptr(A), _ptr(W), _ptr(bias), _ptr(out), _ptr(resid), M, N, K,
+                                          1 if gelu else 0, _ptr(status), _stream_handle(stream)),
+           "enc_linear_bf16")
+    return out if resid is None else resid
+
+
+def attention_bf16(qkv, cu, max_n, n_heads, out=None, stream=None):
+    """Packed-clip bidirectional attention: qkv [R, 3d] bf16, cu device int32 [B+1]."""
+    import torch
+    R = qkv.shape[0]
+    d = 64 * n_heads
+    if out is None:
+        out = torch.empty((R, d), dtype=torch.bfloat16, device=qkv.device)
+    _check(load_library().enc_attention_bf16(_ptr(qkv), _ptr(out), _ptr(cu), int(cu.numel()) - 1, int(max_n),
+                                             int(n_heads), _stream_handle(stream)), "enc_attention_bf16")
+    return out

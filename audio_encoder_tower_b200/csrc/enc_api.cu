@@ -1,0 +1,522 @@
+// C ABI of the encoder tower: argument checks, weight repacking, workspace,
+// tensor maps, and the stream-ordered launch sequence of one forward pass.
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/enc.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace enc;
+
+namespace {
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+inline int round_up(int a, int b) { return ceil_div(a, b) * b; }
+
+struct LayerMaps {
+  CUtensorMap qkv, o, fc1, fc2;
+};
+
+}  // namespace
+
+struct enc_handle {
+  enc_config cfg;
+  int device = 0, sm_count = 0;
+  bool bf16 = true;
+  size_t esz = 2;            // bytes per element of cfg.dtype
+  // geometry
+  int T = 0, Tp = 0, P = 0, P1 = 0, p_out = 0, d_out = 0, mpad = 0;
+  // allocations (all library-owned)
+  std::vector<void*> allocs;
+  size_t bytes = 0;
+  // repacked weights
+  void* conv1_w = nullptr;   // [d, 3, mpad] (bf16) or [d, 3, n_mels] (fp32)
+  void* conv2_w = nullptr;   // [d, 3, d]
+  float *conv1_b = nullptr, *conv2_b = nullptr, *pe = nullptr;
+  std::vector<void*> qkv_w, o_w, fc1_w, fc2_w;                 // per layer
+  std::vector<float*> qkv_b, o_b, fc1_b, fc2_b, ln1_g, ln1_b, ln2_g, ln2_b;
+  float *lnpost_g = nullptr, *lnpost_b = nullptr;
+  void *proj1_w = nullptr, *proj2_w = nullptr;
+  float *proj1_b = nullptr, *proj2_b = nullptr;
+  // workspace
+  void* melT = nullptr;      // [2 + max_batch * Tp, n_mels]; data starts one row in
+  void* y1 = nullptr;        // [max_batch * Tp + 2, d]
+  float* x = nullptr;        // [max_batch * P, d] residual stream
+  void *a = nullptr, *qkv = nullptr, *o = nullptr, *f = nullptr, *e = nullptr, *p1 = nullptr;
+  int* meta = nullptr;       // device [cu (B+1) | cu_out (B+1) | len (B)]
+  int* h_meta = nullptr;     // pinned host staging of meta
+  int* status = nullptr;     // device status word
+  cudaEvent_t meta_free = nullptr;
+  bool meta_pending = false;
+  // tensor maps (bf16 path)
+  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1;
+  CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
+  std::vector<LayerMaps> lmaps;
+};
+
+namespace {
+
+enc_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ENC_OK;
+  if (e == cudaErrorMemoryAllocation) return ENC_ERR_OOM;
+  return ENC_ERR_CUDA;
+}
+
+#define ENC_TRY(expr)                                       \
+  do {                                                      \
+    cudaError_t _e = (expr);                                \
+    if (_e != cudaSuccess) return cuda_status(_e);          \
+  } while (0)
+
+template <typename P>
+enc_status dev_alloc(enc_handle* h, P** out, size_t bytes) {
+  void* p = nullptr;
+  if (bytes == 0) bytes = 16;
+  // Test hook: ENC_FAIL_ALLOC=N makes the N-th allocation (1-based) report failure.
+  static int counter = 0;
+  const char* env = getenv("ENC_FAIL_ALLOC");
+  if (env && atoi(env) > 0 && ++counter == atoi(env)) return ENC_ERR_OOM;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return ENC_ERR_OOM;
+  }
+  h->allocs.push_back(p);
+  h->bytes += bytes;
+  *out = reinterpret_cast<P*>(p);
+  return ENC_OK;
+}
+
+#define ENC_CHECK(expr)                        \
+  do {                                         \
+    enc_status _s = (expr);                    \
+    if (_s != ENC_OK) return _s;               \
+  } while (0)
+
+void free_all(enc_handle* h) {
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+  if (h->h_meta) cudaFreeHost(h->h_meta);
+  h->h_meta = nullptr;
+  if (h->meta_free) cudaEventDestroy(h->meta_free);
+  h->meta_free = nullptr;
+}
+
+enc_status validate_config(const enc_config* c) {
+  if (!c) return ENC_ERR_INVALID_ARG;
+  if (c->flags != 0) return ENC_ERR_INVALID_ARG;
+  if (c->dtype != ENC_DTYPE_BF16 && c->dtype != ENC_DTYPE_FP32) return ENC_ERR_INVALID_ARG;
+  if (c->n_mels <= 0 || c->d_model <= 0 || c->n_layers < 0 || c->n_heads <= 0 || c->ffn_dim <= 0 ||
+      c->max_frames <= 0 || c->max_batch <= 0)
+    return ENC_ERR_INVALID_ARG;
+  if (c->pool_step != 1 && c->pool_step != 2) return ENC_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 || c->n_heads * c->head_dim != c->d_model) return ENC_ERR_UNSUPPORTED;
+  if (c->d_model % 128 || c->d_model > 2048) return ENC_ERR_UNSUPPORTED;
+  if (c->ffn_dim % 128) return ENC_ERR_UNSUPPORTED;
+  if (c->n_mels % 8 || c->n_mels > 256) return ENC_ERR_UNSUPPORTED;
+  if (c->proj_hidden < 0 || c->proj_out < 0) return ENC_ERR_INVALID_ARG;
+  if (c->proj_hidden && (c->proj_hidden % 128 || c->proj_out <= 0 || c->proj_out % 128)) return ENC_ERR_UNSUPPORTED;
+  if (!(c->ln_eps > 0.f)) return ENC_ERR_INVALID_ARG;
+  // index arithmetic stays in 32 bits
+  const long long rows = (long long)c->max_batch * (c->max_frames + 4);
+  if (rows * (long long)(3 * c->d_model > c->ffn_dim ? 3 * c->d_model : c->ffn_dim) > (1ll << 31) - 1)
+    return ENC_ERR_UNSUPPORTED;
+  return ENC_OK;
+}
+
+// Copy `n` elements (cfg dtype) device to device into fresh library memory.
+enc_status copy_weight(enc_handle* h, const void* src, size_t n, void** dst) {
+  if (!src) return ENC_ERR_INVALID_ARG;
+  ENC_CHECK(dev_alloc(h, dst, n * h->esz));
+  ENC_TRY(cudaMemcpy(*dst, src, n * h->esz, cudaMemcpyDeviceToDevice));
+  return ENC_OK;
+}
+
+enc_status to_f32(enc_handle* h, const void* src, int n, float fill, float** dst) {
+  ENC_CHECK(dev_alloc(h, dst, (size_t)n * 4));
+  ENC_TRY(launch_to_f32(src, h->bf16, *dst, n, fill, 0));
+  return ENC_OK;
+}
+
+bool map_rows(CUtensorMap* m, const void* base, int inner, long long rows, int box_rows) {
+  return make_tma_2d(m, base, (uint64_t)inner, (uint64_t)rows, (uint64_t)inner * 2, 64, (uint32_t)box_rows);
+}
+
+enc_status build(enc_handle* h, const enc_weights* w) {
+  const enc_config& c = h->cfg;
+  const int d = c.d_model, F = c.ffn_dim, L = c.n_layers, M = c.n_mels, Bm = c.max_batch;
+  // ---- weights
+  if (!w->conv1_w || !w->conv2_w) return ENC_ERR_INVALID_ARG;
+  h->mpad = h->bf16 ? round_up(M, 64) : M;
+  ENC_CHECK(dev_alloc(h, &h->conv1_w, (size_t)d * 3 * h->mpad * h->esz));
+  ENC_TRY(launch_conv_repack(w->conv1_w, h->bf16, h->conv1_w, h->bf16, d, M, h->mpad, 0));
+  ENC_CHECK(dev_alloc(h, &h->conv2_w, (size_t)d * 3 * d * h->esz));
+  ENC_TRY(launch_conv_repack(w->conv2_w, h->bf16, h->conv2_w, h->bf16, d, d, d, 0));
+  ENC_CHECK(to_f32(h, w->conv1_b, d, 0.f, &h->conv1_b));
+  ENC_CHECK(to_f32(h, w->conv2_b, d, 0.f, &h->conv2_b));
+  if (L > 0 && (!w->ln1_g || !w->ln1_b || !w->q_w || !w->q_b || !w->k_w || !w->v_w || !w->v_b || !w->o_w ||
+                !w->o_b || !w->ln2_g || !w->ln2_b || !w->fc1_w || !w->fc1_b || !w->fc2_w || !w->fc2_b))
+    return ENC_ERR_INVALID_ARG;
+  h->qkv_w.resize(L); h->o_w.resize(L); h->fc1_w.resize(L); h->fc2_w.resize(L);
+  h->qkv_b.resize(L); h->o_b.resize(L); h->fc1_b.resize(L); h->fc2_b.resize(L);
+  h->ln1_g.resize(L); h->ln1_b.resize(L); h->ln2_g.resize(L); h->ln2_b.resize(L);
+  const size_t dd = (size_t)d * d;
+  for (int l = 0; l < L; ++l) {
+    if (!w->q_w[l] || !w->k_w[l] || !w->v_w[l] || !w->o_w[l] || !w->fc1_w[l] || !w->fc2_w[l])
+      return ENC_ERR_INVALID_ARG;
+    ENC_CHECK(dev_alloc(h, &h->qkv_w[l], 3 * dd * h->esz));
+    uint8_t* q = reinterpret_cast<uint8_t*>(h->qkv_w[l]);
+    ENC_TRY(cudaMemcpy(q, w->q_w[l], dd * h->esz, cudaMemcpyDeviceToDevice));
+    ENC_TRY(cudaMemcpy(q + dd * h->esz, w->k_w[l], dd * h->esz, cudaMemcpyDeviceToDevice));
+    ENC_TRY(cudaMemcpy(q + 2 * dd * h->esz, w->v_w[l], dd * h->esz, cudaMemcpyDeviceToDevice));
+    ENC_CHECK(dev_alloc(h, &h->qkv_b[l], 3 * (size_t)d * 4));
+    ENC_TRY(launch_to_f32(w->q_b[l], h->bf16, h->qkv_b[l], d, 0.f, 0));
+    // a key bias shifts every score of a query row equally and cancels in softmax: k runs unbiased
+    ENC_TRY(launch_to_f32(nullptr, h->bf16, h->qkv_b[l] + d, d, 0.f, 0));
+    ENC_TRY(launch_to_f32(w->v_b[l], h->bf16, h->qkv_b[l] + 2 * d, d, 0.f, 0));
+    ENC_CHECK(copy_weight(h, w->o_w[l], dd, &h->o_w[l]));
+    ENC_CHECK(copy_weight(h, w->fc1_w[l], (size_t)F * d, &h->fc1_w[l]));
+    ENC_CHECK(copy_weight(h, w->fc2_w[l], (size_t)d * F, &h->fc2_w[l]));
+    ENC_CHECK(to_f32(h, w->o_b[l], d, 0.f, &h->o_b[l]));
+    ENC_CHECK(to_f32(h, w->fc1_b[l], F, 0.f, &h->fc1_b[l]));
+    ENC_CHECK(to_f32(h, w->fc2_b[l], d, 0.f, &h->fc2_b[l]));
+    ENC_CHECK(to_f32(h, w->ln1_g[l], d, 1.f, &h->ln1_g[l]));
+    ENC_CHECK(to_f32(h, w->ln1_b[l], d, 0.f, &h->ln1_b[l]));
+    ENC_CHECK(to_f32(h, w->ln2_g[l], d, 1.f, &h->ln2_g[l]));
+    ENC_CHECK(to_f32(h, w->ln2_b[l], d, 0.f, &h->ln2_b[l]));
+  }
+  ENC_CHECK(to_f32(h, w->lnpost_g, d, 1.f, &h->lnpost_g));
+  ENC_CHECK(to_f32(h, w->lnpost_b, d, 0.f, &h->lnpost_b));
+  const int ph = c.proj_hidden, po = c.proj_out;
+  if (ph) {
+    ENC_CHECK(copy_weight(h, w->proj1_w, (size_t)ph * d, &h->proj1_w));
+    ENC_CHECK(copy_weight(h, w->proj2_w, (size_t)po * ph, &h->proj2_w));
+    ENC_CHECK(to_f32(h, w->proj1_b, ph, 0.f, &h->proj1_b));
+    ENC_CHECK(to_f32(h, w->proj2_b, po, 0.f, &h->proj2_b));
+  }
+  // ---- position table
+  ENC_CHECK(dev_alloc(h, &h->pe, (size_t)h->P * d * 4));
+  ENC_TRY(launch_position_table(h->pe, h->P, d, 0));
+  // ---- workspace
+  const long long rows_t = (long long)Bm * h->Tp, rows_p = (long long)Bm * h->P, rows_o = (long long)Bm * h->p_out;
+  ENC_CHECK(dev_alloc(h, &h->melT, (size_t)(rows_t + 2) * M * h->esz));
+  ENC_CHECK(dev_alloc(h, &h->y1, (size_t)(rows_t + 2) * d * h->esz));
+  ENC_TRY(cudaMemset(h->melT, 0, (size_t)(rows_t + 2) * M * h->esz));
+  ENC_TRY(cudaMemset(h->y1, 0, (size_t)(rows_t + 2) * d * h->esz));
+  ENC_CHECK(dev_alloc(h, &h->x, (size_t)rows_p * d * 4));
+  ENC_CHECK(dev_alloc(h, &h->a, (size_t)rows_p * d * h->esz));
+  ENC_CHECK(dev_alloc(h, &h->qkv, (size_t)rows_p * 3 * d * h->esz));
+  ENC_CHECK(dev_alloc(h, &h->o, (size_t)rows_p * d * h->esz));
+  ENC_CHECK(dev_alloc(h, &h->f, (size_t)rows_p * F * h->esz));
+  if (ph) {
+    ENC_CHECK(dev_alloc(h, &h->e, (size_t)rows_o * d * h->esz));
+    ENC_CHECK(dev_alloc(h, &h->p1, (size_t)rows_o * ph * h->esz));
+  }
+  ENC_CHECK(dev_alloc(h, &h->meta, (size_t)(3 * Bm + 2) * 4));
+  ENC_CHECK(dev_alloc(h, &h->status, 4));
+  ENC_TRY(cudaMemset(h->status, 0, 4));
+  if (cudaMallocHost(&h->h_meta, (size_t)(3 * Bm + 2) * 4) != cudaSuccess) {
+    cudaGetLastError();
+    h->h_meta = nullptr;
+    return ENC_ERR_OOM;
+  }
+  ENC_TRY(cudaEventCreateWithFlags(&h->meta_free, cudaEventDisableTiming));
+  // ---- tensor maps (tensor-core path)
+  if (h->bf16) {
+    const uint8_t* melT_data = reinterpret_cast<const uint8_t*>(h->melT) + (size_t)M * 2;
+    bool ok = map_rows(&h->m_conv1_a, melT_data, M, rows_t, 128);
+    ok = ok && make_tma_2d(&h->m_conv2_a, h->y1, 2 * (uint64_t)d, (uint64_t)rows_t / 2, 4 * (uint64_t)d, 64, 128);
+    ok = ok && map_rows(&h->m_a, h->a, d, rows_p, 128);
+    ok = ok && map_rows(&h->m_o, h->o, d, rows_p, 128);
+    ok = ok && map_rows(&h->m_f, h->f, F, rows_p, 128);
+    ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
+    ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
+    if (ph) {
+      ok = ok && map_rows(&h->m_e, h->e, d, rows_o, 128);
+      ok = ok && map_rows(&h->m_p1, h->p1, ph, rows_o, 128);
+      ok = ok && map_rows(&h->m_proj1_w, h->proj1_w, d, ph, gemm_tile_n(ph));
+      ok = ok && map_rows(&h->m_proj2_w, h->proj2_w, ph, po, gemm_tile_n(po));
+    }
+    h->lmaps.resize(L);
+    for (int l = 0; ok && l < L; ++l) {
+      ok = ok && map_rows(&h->lmaps[l].qkv, h->qkv_w[l], d, 3 * d, gemm_tile_n(3 * d));
+      ok = ok && map_rows(&h->lmaps[l].o, h->o_w[l], d, d, gemm_tile_n(d));
+      ok = ok && map_rows(&h->lmaps[l].fc1, h->fc1_w[l], d, F, gemm_tile_n(F));
+      ok = ok && map_rows(&h->lmaps[l].fc2, h->fc2_w[l], F, d, gemm_tile_n(d));
+    }
+    if (!ok) return ENC_ERR_CUDA;
+  }
+  ENC_TRY(cudaDeviceSynchronize());
+  return ENC_OK;
+}
+
+EpiParams epi_base(int mode) {
+  EpiParams e;
+  memset(&e, 0, sizeof(e));
+  e.mode = mode;
+  return e;
+}
+
+// ------------------------------------------------------------- forward (bf16)
+enc_status forward_bf16(enc_handle* h, const void* mel, int B, void* out, int R, int R_out, int max_n,
+                        cudaStream_t s) {
+  const enc_config& c = h->cfg;
+  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
+  const int* cu = h->meta;
+  const int* cu_out = h->meta + (B + 1);
+  const int* len = h->meta + 2 * (B + 1);
+  bf16* melT_data = reinterpret_cast<bf16*>(h->melT) + M;
+  ENC_TRY(launch_mel_stage<bf16>(reinterpret_cast<const bf16*>(mel), len, melT_data, B, M, h->T, h->Tp, s));
+
+  GemmTcParams g;
+  memset(&g, 0, sizeof(g));
+  g.status = h->status;
+  // conv1: rows = padded time of every clip
+  g.M = B * h->Tp; g.N = d; g.a_mode = A_CONV1; g.kb_seg = h->mpad / 64; g.num_kb = 3 * g.kb_seg;
+  g.epi = epi_base(EPI_CONV1);
+  g.epi.bias = h->conv1_b; g.epi.out = h->y1; g.epi.ldo = d; g.epi.T = h->T; g.epi.Tp = h->Tp;
+  ENC_TRY(launch_gemm_tc(h->m_conv1_a, h->m_conv1_w, g, h->sm_count, s));
+  // conv2 (+ GELU + position table) -> packed residual stream
+  g.M = B * h->P1; g.N = d; g.a_mode = A_CONV2; g.kb_seg = d / 64; g.num_kb = 3 * g.kb_seg;
+  g.epi = epi_base(EPI_CONV2);
+  g.epi.bias = h->conv2_b; g.epi.resid = h->x; g.epi.ldo = d; g.epi.pe = h->pe; g.epi.cu = cu; g.epi.P1 = h->P1;
+  ENC_TRY(launch_gemm_tc(h->m_conv2_a, h->m_conv2_w, g, h->sm_count, s));
+
+  for (int l = 0; l < c.n_layers; ++l) {
+    const LayerMaps& lm = h->lmaps[l];
+    ENC_TRY(launch_layernorm<bf16>(h->x, h->ln1_g[l], h->ln1_b[l], reinterpret_cast<bf16*>(h->a), R, d, c.ln_eps, s));
+    g.M = R; g.a_mode = A_PLAIN; g.kb_seg = 0;
+    g.N = 3 * d; g.num_kb = d / 64;
+    g.epi = epi_base(EPI_STORE);
+    g.epi.bias = h->qkv_b[l]; g.epi.out = h->qkv; g.epi.ldo = 3 * d;
+    ENC_TRY(launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s));
+    ENC_TRY(launch_attention_bf16(reinterpret_cast<const bf16*>(h->qkv), reinterpret_cast<bf16*>(h->o), cu, B, max_n,
+                                  d, c.n_heads, s));
+    g.N = d; g.num_kb = d / 64;
+    g.epi = epi_base(EPI_RESIDUAL);
+    g.epi.bias = h->o_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
+    ENC_TRY(launch_gemm_tc(h->m_o, lm.o, g, h->sm_count, s));
+    ENC_TRY(launch_layernorm<bf16>(h->x, h->ln2_g[l], h->ln2_b[l], reinterpret_cast<bf16*>(h->a), R, d, c.ln_eps, s));
+    g.N = F; g.num_kb = d / 64;
+    g.epi = epi_base(EPI_STORE);
+    g.epi.gelu = 1; g.epi.bias = h->fc1_b[l]; g.epi.out = h->f; g.epi.ldo = F;
+    ENC_TRY(launch_gemm_tc(h->m_a, lm.fc1, g, h->sm_count, s));
+    g.N = d; g.num_kb = F / 64;
+    g.epi = epi_base(EPI_RESIDUAL);
+    g.epi.bias = h->fc2_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
+    ENC_TRY(launch_gemm_tc(h->m_f, lm.fc2, g, h->sm_count, s));
+  }
+
+  if (!c.proj_hidden) {
+    ENC_TRY(launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(out), B,
+                                  h->p_out, d, c.pool_step, 0, c.ln_eps, s));
+    return ENC_OK;
+  }
+  const int ph = c.proj_hidden, po = c.proj_out;
+  ENC_TRY(launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(h->e), B,
+                                h->p_out, d, c.pool_step, 1, c.ln_eps, s));
+  g.M = R_out; g.a_mode = A_PLAIN; g.kb_seg = 0;
+  g.N = ph; g.num_kb = d / 64;
+  g.epi = epi_base(EPI_STORE);
+  g.epi.gelu = 1; g.epi.bias = h->proj1_b; g.epi.out = h->p1; g.epi.ldo = ph;
+  ENC_TRY(launch_gemm_tc(h->m_e, h->m_proj1_w, g, h->sm_count, s));
+  g.N = po; g.num_kb = ph / 64;
+  g.epi = epi_base(EPI_SCATTER);
+  g.epi.bias = h->proj2_b; g.epi.out = out; g.epi.ldo = po; g.epi.cu = cu_out; g.epi.B = B; g.epi.p_out = h->p_out;
+  ENC_TRY(launch_gemm_tc(h->m_p1, h->m_proj2_w, g, h->sm_count, s));
+  ENC_TRY(launch_zero_tail_rows<bf16>(reinterpret_cast<bf16*>(out), cu_out, B, h->p_out, po, s));
+  return ENC_OK;
+}
+
+// -------------------------------------------------------- forward (fp32 check)
+enc_status forward_f32(enc_handle* h, const void* mel, int B, void* out, int R, int R_out, int max_n,
+                       cudaStream_t s) {
+  const enc_config& c = h->cfg;
+  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
+  const int* cu = h->meta;
+  const int* cu_out = h->meta + (B + 1);
+  const int* len = h->meta + 2 * (B + 1);
+  float* melT = reinterpret_cast<float*>(h->melT);
+  float* y1 = reinterpret_cast<float*>(h->y1);
+  ENC_TRY(launch_mel_stage<float>(reinterpret_cast<const float*>(mel), len, melT + M, B, M, h->T, h->Tp, s));
+
+  EpiParams e = epi_base(EPI_CONV1);
+  e.bias = h->conv1_b; e.out = y1; e.ldo = d; e.T = h->T; e.Tp = h->Tp;
+  // conv1 row r reads mel rows r-1, r, r+1: A starts at the guard row, rows overlap (lda = M)
+  ENC_TRY(launch_sgemm(melT, M, reinterpret_cast<const float*>(h->conv1_w), 3 * M, B * h->Tp, d, 3 * M, e, s));
+  e = epi_base(EPI_CONV2);
+  e.bias = h->conv2_b; e.resid = h->x; e.ldo = d; e.pe = h->pe; e.cu = cu; e.P1 = h->P1;
+  // conv2 row j reads conv1 rows 2j, 2j+1, 2j+2 (padded time): lda = 2d, K = 3d
+  ENC_TRY(launch_sgemm(y1, 2 * d, reinterpret_cast<const float*>(h->conv2_w), 3 * d, B * h->P1, d, 3 * d, e, s));
+
+  float* a = reinterpret_cast<float*>(h->a);
+  float* qkv = reinterpret_cast<float*>(h->qkv);
+  float* o = reinterpret_cast<float*>(h->o);
+  float* f = reinterpret_cast<float*>(h->f);
+  for (int l = 0; l < c.n_layers; ++l) {
+    ENC_TRY(launch_layernorm<float>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
+    e = epi_base(EPI_STORE);
+    e.bias = h->qkv_b[l]; e.out = qkv; e.ldo = 3 * d;
+    ENC_TRY(launch_sgemm(a, d, reinterpret_cast<const float*>(h->qkv_w[l]), d, R, 3 * d, d, e, s));
+    ENC_TRY(launch_attention_f32(qkv, o, cu, B, max_n, d, c.n_heads, s));
+    e = epi_base(EPI_RESIDUAL);
+    e.bias = h->o_b[l]; e.resid = h->x; e.ldo = d;
+    ENC_TRY(launch_sgemm(o, d, reinterpret_cast<const float*>(h->o_w[l]), d, R, d, d, e, s));
+    ENC_TRY(launch_layernorm<float>(h->x, h->ln2_g[l], h->ln2_b[l], a, R, d, c.ln_eps, s));
+    e = epi_base(EPI_STORE);
+    e.gelu = 1; e.bias = h->fc1_b[l]; e.out = f; e.ldo = F;
+    ENC_TRY(launch_sgemm(a, d, reinterpret_cast<const float*>(h->fc1_w[l]), d, R, F, d, e, s));
+    e = epi_base(EPI_RESIDUAL);
+    e.bias = h->fc2_b[l]; e.resid = h->x; e.ldo = d;
+    ENC_TRY(launch_sgemm(f, F, reinterpret_cast<const float*>(h->fc2_w[l]), F, R, d, F, e, s));
+  }
+  if (!c.proj_hidden) {
+    ENC_TRY(launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<float*>(out), B,
+                                   h->p_out, d, c.pool_step, 0, c.ln_eps, s));
+    return ENC_OK;
+  }
+  const int ph = c.proj_hidden, po = c.proj_out;
+  float* ev = reinterpret_cast<float*>(h->e);
+  float* p1 = reinterpret_cast<float*>(h->p1);
+  ENC_TRY(launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, ev, B, h->p_out, d, c.pool_step, 1,
+                                 c.ln_eps, s));
+  e = epi_base(EPI_STORE);
+  e.gelu = 1; e.bias = h->proj1_b; e.out = p1; e.ldo = ph;
+  ENC_TRY(launch_sgemm(ev, d, reinterpret_cast<const float*>(h->proj1_w), d, R_out, ph, d, e, s));
+  e = epi_base(EPI_SCATTER);
+  e.bias = h->proj2_b; e.out = out; e.ldo = po; e.cu = cu_out; e.B = B; e.p_out = h->p_out;
+  ENC_TRY(launch_sgemm(p1, ph, reinterpret_cast<const float*>(h->proj2_w), ph, R_out, po, ph, e, s));
+  ENC_TRY(launch_zero_tail_rows<float>(reinterpret_cast<float*>(out), cu_out, B, h->p_out, po, s));
+  return ENC_OK;
+}
+
+int valid_out(const enc_handle* h, int n) { return h->cfg.pool_step > 1 ? n / h->cfg.pool_step : n; }
+
+}  // namespace
+
+extern "C" {
+
+const char* enc_status_string(enc_status s) {
+  switch (s) {
+    case ENC_OK: return "ok";
+    case ENC_ERR_INVALID_ARG: return "invalid argument";
+    case ENC_ERR_UNSUPPORTED: return "unsupported geometry or device (needs sm_100)";
+    case ENC_ERR_OOM: return "out of memory";
+    case ENC_ERR_CUDA: return "CUDA runtime error";
+    case ENC_ERR_TIMEOUT: return "device-side wait timed out";
+    case ENC_ERR_DEVICE_CHECK: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+enc_status enc_create(const enc_config* cfg, const enc_weights* w, enc_handle** out) {
+  if (!out) return ENC_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!w) return ENC_ERR_INVALID_ARG;
+  enc_status st = validate_config(cfg);
+  if (st != ENC_OK) return st;
+  int dev = 0;
+  cudaDeviceProp prop;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ENC_ERR_CUDA;
+  }
+  if (prop.major != 10 || prop.minor != 0) return ENC_ERR_UNSUPPORTED;
+  enc_handle* h = new enc_handle();
+  h->cfg = *cfg;
+  h->device = dev;
+  h->sm_count = prop.multiProcessorCount;
+  h->bf16 = cfg->dtype == ENC_DTYPE_BF16;
+  h->esz = h->bf16 ? 2 : 4;
+  h->T = cfg->max_frames;
+  h->Tp = round_up(h->T + 2, 2);
+  h->P = (h->T + 1) / 2;
+  h->P1 = h->P + 1;
+  h->p_out = cfg->pool_step > 1 ? h->P / cfg->pool_step : h->P;
+  h->d_out = cfg->proj_hidden ? cfg->proj_out : cfg->d_model;
+  st = build(h, w);
+  if (st != ENC_OK) {
+    cudaDeviceSynchronize();
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return st;
+  }
+  *out = h;
+  return ENC_OK;
+}
+
+enc_status enc_output_positions(const enc_handle* h, int32_t B, const int32_t* lengths, int32_t* n_out,
+                                int32_t* p_out, int32_t* d_out) {
+  if (!h || B < 1) return ENC_ERR_INVALID_ARG;
+  if (n_out) {
+    for (int b = 0; b < B; ++b) {
+      const int len = lengths ? lengths[b] : h->T;
+      if (len < 1 || len > h->T) return ENC_ERR_INVALID_ARG;
+      n_out[b] = valid_out(h, (len + 1) / 2);
+    }
+  }
+  if (p_out) *p_out = h->p_out;
+  if (d_out) *d_out = h->d_out;
+  return ENC_OK;
+}
+
+enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, int32_t B, void* out,
+                       cudaStream_t stream) {
+  if (!h || !mel || !out || B < 1 || B > h->cfg.max_batch) return ENC_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(mel) | reinterpret_cast<uintptr_t>(out)) & 15u) return ENC_ERR_INVALID_ARG;
+  // per-clip counts (host): n_b = ceil(len_b / 2) positions, packed offsets
+  std::vector<int> len(B), cu(B + 1), cu_out(B + 1);
+  int max_n = 0;
+  cu[0] = cu_out[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    len[b] = lengths ? lengths[b] : h->T;
+    if (len[b] < 1 || len[b] > h->T) return ENC_ERR_INVALID_ARG;
+    const int n = (len[b] + 1) / 2;
+    cu[b + 1] = cu[b] + n;
+    cu_out[b + 1] = cu_out[b] + valid_out(h, n);
+    if (n > max_n) max_n = n;
+  }
+  if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
+  // the pinned staging buffer may still feed the previous forward's upload
+  if (h->meta_pending) ENC_TRY(cudaEventSynchronize(h->meta_free));
+  int* hm = h->h_meta;
+  memcpy(hm, cu.data(), (B + 1) * 4);
+  memcpy(hm + B + 1, cu_out.data(), (B + 1) * 4);
+  memcpy(hm + 2 * (B + 1), len.data(), B * 4);
+  ENC_TRY(cudaMemcpyAsync(h->meta, hm, (size_t)(3 * B + 2) * 4, cudaMemcpyHostToDevice, stream));
+  ENC_TRY(cudaEventRecord(h->meta_free, stream));
+  h->meta_pending = true;
+  const int R = cu[B], R_out = cu_out[B];
+  return h->bf16 ? forward_bf16(h, mel, B, out, R, R_out, max_n, stream)
+                 : forward_f32(h, mel, B, out, R, R_out, max_n, stream);
+}
+
+enc_status enc_get_status(enc_handle* h, cudaStream_t stream) {
+  if (!h) return ENC_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  int v = 0;
+  ENC_TRY(cudaMemcpy(&v, h->status, 4, cudaMemcpyDeviceToHost));
+  if (v != 0) ENC_TRY(cudaMemset(h->status, 0, 4));
+  if (v == kDevTimeout) return ENC_ERR_TIMEOUT;
+  if (v == kDevCheck) return ENC_ERR_DEVICE_CHECK;
+  return v == 0 ? ENC_OK : ENC_ERR_CUDA;
+}
+
+void enc_destroy(enc_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+}
+
+size_t enc_device_bytes(const enc_handle* h) { return h ? h->bytes : 0; }
+
+}  // extern "C"

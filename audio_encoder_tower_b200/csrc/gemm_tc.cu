@@ -1,0 +1,262 @@
+// tcgen05 (UMMA) GEMM with fused epilogues for the encoder's dense contractions:
+//   conv1 / conv2 (implicit GEMM over TMA-staged taps), QKV, out-proj, fc1, fc2,
+//   projector fc1 / fc2.
+//
+//   C[M, N] = A[M, K] * W[N, K]^T, bf16 operands, fp32 accumulation in TMEM.
+//
+// Design (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: 64-wide K slices of A (128 rows) and W (BN rows)
+//               into a kStages-deep shared-memory ring, 128-byte swizzle.
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16)
+//               into a double-buffered TMEM accumulator (2 x BN columns) and
+//               frees ring slots / publishes finished tiles with tcgen05.commit.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (one row per thread),
+//               apply bias / GELU / residual / position-table / scatter, store.
+// The epilogue of tile i overlaps the MMAs of tile i+1.
+//
+// The A operand of the convolutions is never materialised as an im2col matrix:
+//   conv1: tap k of output row r is row r + k - 1 of the time-major mel buffer
+//          (a shifted TMA box; row -1 and rows past the end read as zeros);
+//   conv2: the conv1 output [rows, d] is viewed as [rows/2, 2d] ("pairs");
+//          output j needs pair j (taps 0, 1) and the first half of pair j + 1.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace enc {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any legitimate wait
+
+template <int BN>
+struct TcCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr uint32_t kABytes = BM * BK * 2;
+  static constexpr uint32_t kBBytes = BN * BK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTmemCols = 2 * BN;
+  static constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * (size_t)kStageBytes + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, int& x, int& y) {
+  if (p.a_mode == A_CONV1) {
+    const int tap = kb / p.kb_seg;
+    x = (kb - tap * p.kb_seg) * BK;
+    y = m0 + tap - 1;
+  } else if (p.a_mode == A_CONV2) {
+    if (kb < 2 * p.kb_seg) { x = kb * BK; y = m0; }
+    else { x = (kb - 2 * p.kb_seg) * BK; y = m0 + 1; }
+  } else {
+    x = kb * BK;
+    y = m0;
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+               const GemmTcParams p) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;    // [2] accumulator ready
+  uint64_t* tempty = tfull + 2;            // [2] accumulator drained
+  uint64_t* drain = tempty + 2;            // all MMAs of this CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiWarps * 32); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&map_a); tma_prefetch_desc(&map_b); }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t armed = 0, armed_phase = 0;   // bit s: slot s holds a load; its phase parity
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          int ax, ay;
+          a_coords(p, m0, kb, ax, ay);
+          tma_load_2d(sA + stage * C::kABytes, &map_a, &full[stage], ax, ay);
+          tma_load_2d(sB + stage * C::kBBytes, &map_b, &full[stage], kb * BK, n0);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        set_status(p.status, kDevTimeout);
+        *abort_v = 1;
+        // let copies already in flight land before the CTA's shared memory goes away
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * C::kABytes));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * C::kBBytes));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K inside the swizzled row
+            umma_f16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k), idesc,
+                        (kb | k) != 0 ? 1u : 0u);
+          issued = true;
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) { set_status(p.status, kDevTimeout); *abort_v = 1; }
+      if (issued) {   // every MMA done before TMEM is released
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, kWaitLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;          // TMEM lanes this warp may read: 32*quarter ..
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
+        set_status(p.status, kDevTimeout);
+        *abort_v = 1;
+        break;
+      }
+      tc_fence_after();
+      const int r = m0 + quarter * 32 + lane;
+      int dst = 0, pe_row = 0;
+      bool zero = false;
+      const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+        tmem_wait_ld();
+        if (row_ok) epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+template <int BN>
+bool configure_once() {
+  static unsigned long long done = 0;   // bit per device ordinal
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(done & bit)) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)TcCfg<BN>::kSmemBytes) != cudaSuccess)
+      return false;
+    done |= bit;
+  }
+  return true;
+}
+
+}  // namespace
+
+int gemm_tile_n(int n) { return (n % 256 == 0) ? 256 : 128; }
+
+bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
+                 uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn || !base) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (pitch_bytes & 15u)) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
+                           cudaStream_t stream) {
+  if (p.M <= 0) return cudaSuccess;
+  const int bn = gemm_tile_n(p.N);
+  p.tiles_n = p.N / bn;
+  p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
+  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+  if (bn == 256) {
+    if (!configure_once<256>()) return cudaErrorInvalidValue;
+    gemm_tc_kernel<256><<<grid, kThreads, TcCfg<256>::kSmemBytes, stream>>>(map_a, map_b, p);
+  } else {
+    if (!configure_once<128>()) return cudaErrorInvalidValue;
+    gemm_tc_kernel<128><<<grid, kThreads, TcCfg<128>::kSmemBytes, stream>>>(map_a, map_b, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace enc

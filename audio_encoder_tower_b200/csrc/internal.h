@@ -1,0 +1,77 @@
+// Launchers shared between the kernel files and the C-ABI layer (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace enc {
+
+// ----------------------------------------------------------- tcgen05 GEMM
+enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2 };
+
+struct GemmTcParams {
+  int M, N;        // output rows / columns (N a multiple of 128)
+  int num_kb;      // K / 64
+  int a_mode;      // AMode
+  int kb_seg;      // k-blocks per tap segment (conv modes)
+  int tiles_n;     // filled by the launcher
+  int num_tiles;   // filled by the launcher
+  EpiParams epi;
+  int* status;
+};
+
+int gemm_tile_n(int n);   // 256 when N % 256 == 0, else 128
+
+// 2-D bf16 tensor map with 128-byte swizzle and zero fill outside the tensor.
+bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
+                 uint32_t box_inner, uint32_t box_rows);
+
+cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
+                           cudaStream_t stream);
+
+// --------------------------------------------------------- fp32 check path
+// C = A[M, K] (row stride lda, rows may overlap) * W[N, K]^T (row stride ldw).
+cudaError_t launch_sgemm(const float* A, int lda, const float* W, int ldw, int M, int N, int K, const EpiParams& e,
+                         cudaStream_t stream);
+
+// ------------------------------------------------------------- attention
+// qkv [R, 3d] packed rows (clip b at rows cu[b] .. cu[b+1]); out [R, d].
+cudaError_t launch_attention_bf16(const bf16* qkv, bf16* out, const int* cu, int B, int max_n, int d, int H,
+                                  cudaStream_t stream);
+cudaError_t launch_attention_f32(const float* qkv, float* out, const int* cu, int B, int max_n, int d, int H,
+                                 cudaStream_t stream);
+
+// ------------------------------------------------------------- row kernels
+// mel [B, M, T] (clip-major) -> time-major rows [B * Tp, M]: row b*Tp + tp holds
+// frame tp - 1 (zero for tp == 0, tp > T and frames >= len[b]).
+template <typename T>
+cudaError_t launch_mel_stage(const T* mel, const int* len, T* dst, int B, int M, int Tfr, int Tp, cudaStream_t s);
+
+// y = LN(x) * g + b per row; x fp32 [rows, d].
+template <typename OutT>
+cudaError_t launch_layernorm(const float* x, const float* g, const float* b, OutT* y, int rows, int d, float eps,
+                             cudaStream_t s);
+
+// Final LN (+ average pool over `pool` consecutive rows) of packed rows.
+// packed == 0: out is [B, p_out, d] with zero rows past each clip's valid count.
+// packed == 1: out holds only the valid rows, at cu_out[b] + j.
+template <typename OutT>
+cudaError_t launch_final_ln(const float* x, const float* g, const float* b, const int* cu, const int* cu_out,
+                            OutT* out, int B, int p_out, int d, int pool, int packed, float eps, cudaStream_t s);
+
+// Zero rows j >= cu_out[b+1] - cu_out[b] of out [B, p_out, width].
+template <typename OutT>
+cudaError_t launch_zero_tail_rows(OutT* out, const int* cu_out, int B, int p_out, int width, cudaStream_t s);
+
+// ------------------------------------------------------------ set-up work
+cudaError_t launch_position_table(float* pe, int P, int d, cudaStream_t s);
+// src [rows, C, 3] (dtype of src) -> dst [rows, 3, cpad] (dtype of dst), zero padded.
+cudaError_t launch_conv_repack(const void* src, bool src_bf16, void* dst, bool dst_bf16, int rows, int C, int cpad,
+                               cudaStream_t s);
+// n values of src (bf16 or fp32; nullptr -> fill) to fp32.
+cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, int n, float fill, cudaStream_t s);
+
+}  // namespace enc

@@ -1,0 +1,78 @@
+"""Single-kernel parity on the GPU: the tcgen05 linear layer and the flash
+attention kernel against the oracle's float64 steps (same bf16 inputs)."""
+import numpy as np
+import pytest
+
+import oracle as O
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+RNG = np.random.default_rng(7)
+
+
+def _bf16(a):
+    return S.round_bf16(np.asarray(a, np.float32))
+
+
+def _dev(a, dtype=None):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype or torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (127, 256, 128), (128, 384, 64), (300, 1280, 1280),
+                                   (1000, 512, 320), (4000, 3840, 1280)])
+@pytest.mark.parametrize("gelu", [False, True])
+def test_linear_bf16(M, N, K, gelu):
+    import torch
+    from audio_encoder_tower_b200.binding import linear_bf16
+    A = _bf16(RNG.standard_normal((M, K)))
+    W = _bf16(RNG.standard_normal((N, K)) * 0.05)
+    b = RNG.standard_normal(N).astype(np.float32) * 0.1
+    out = linear_bf16(_dev(A), _dev(W), _dev(b, torch.float32), gelu=gelu)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = O.linear(A, W, b)
+    if gelu:
+        ref = O.gelu(ref)
+    err = np.abs(got - ref)
+    assert np.all(err <= 8e-3 * np.maximum(1.0, np.abs(ref))), float(err.max())
+
+
+@pytest.mark.parametrize("M,N,K", [(77, 256, 64), (513, 1280, 5120)])
+def test_linear_residual(M, N, K):
+    import torch
+    from audio_encoder_tower_b200.binding import linear_bf16
+    A = _bf16(RNG.standard_normal((M, K)))
+    W = _bf16(RNG.standard_normal((N, K)) * 0.02)
+    b = RNG.standard_normal(N).astype(np.float32)
+    x0 = RNG.standard_normal((M, N)).astype(np.float32)
+    x = _dev(x0, torch.float32)
+    linear_bf16(_dev(A), _dev(W), _dev(b, torch.float32), resid=x)
+    torch.cuda.synchronize()
+    got = x.cpu().numpy().astype(np.float64)
+    ref = x0 + O.linear(A, W, b)
+    assert np.abs(got - ref).max() < 1e-4 * max(1.0, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("lengths,heads,qscale", [([1, 77, 300], 2, 1.0), ([64, 128, 129], 1, 1.0),
+                                                  ([1500], 3, 1.0), ([200, 513], 2, 6.0)])
+def test_attention_bf16(lengths, heads, qscale):
+    import torch
+    from audio_encoder_tower_b200.binding import attention_bf16
+    d = 64 * heads
+    R = sum(lengths)
+    q = _bf16(RNG.standard_normal((R, d)) * qscale)
+    k = _bf16(RNG.standard_normal((R, d)))
+    v = _bf16(RNG.standard_normal((R, d)))
+    qkv = np.concatenate([q, k, v], axis=1)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    out = attention_bf16(_dev(qkv), _dev(cu, torch.int32), max(lengths), heads)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    for b, n in enumerate(lengths):
+        s = slice(cu[b], cu[b + 1])
+        ref = O.attention(q[s], k[s], v[s], heads, n)
+        err = np.abs(got[s] - ref)
+        # bf16 probabilities and bf16 output: a few 2^-8 of the value range
+        assert err.max() < 3e-2, (b, float(err.max()))
+        assert np.linalg.norm(got[s] - ref) / np.linalg.norm(ref) < 1e-2

@@ -1,0 +1,134 @@
+"""Encoder parity on the GPU through the C ABI against the CPU oracle.
+
+Small cases run whole (every clip, every row) and span several 128-row tiles
+with ragged tails; the full-size workloads run in the configuration the
+benchmark times and are checked on sampled clips (clips are independent, so a
+sampled clip's oracle output is exact for its rows of the batch)."""
+import numpy as np
+import pytest
+
+import oracle as O
+import synthetic as S
+from tests.encoder_cases import assert_parity, compare, make_encoder, oracle_clip, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(name, **kw):
+    base = dict(name=name, n_mels=80, d_model=256, n_layers=2, n_heads=4, ffn_dim=512, frames=333, batch=3,
+                dtype="bf16", seed=11)
+    base.update(kw)
+    return S.EncoderConfig(**base)
+
+
+SMALL = [
+    (_small("small_ragged"), [333, 200, 1]),
+    (_small("small_even", frames=400, n_mels=128), [400, 399, 256]),
+    (_small("small_pool", pool_step=2, frames=301), [301, 300, 7]),
+    (_small("small_proj", proj_hidden=384, proj_out=256), [333, 129, 2]),
+    (_small("small_pool_proj", pool_step=2, proj_hidden=256, proj_out=384, d_model=384, n_heads=6), [333, 50, 3]),
+    (_small("small_fp32", dtype="fp32"), [333, 200, 1]),
+    (_small("small_fp32_pool_proj", dtype="fp32", pool_step=2, proj_hidden=256, proj_out=128), [333, 31, 4]),
+    (_small("peaky", weight_std=0.2, frames=260), [260, 131, 65]),
+]
+
+
+def _run_case(cfg, lengths):
+    w = S.make_weights(cfg)
+    mel = S.make_mel(cfg)
+    enc = make_encoder(cfg, to_device(cfg, w))
+    got = run_gpu(enc, cfg, mel, lengths)
+    n_out, p_out, d_out = enc.output_positions(cfg.batch, lengths)
+    enc.close()
+    return w, mel, got, n_out, p_out, d_out
+
+
+@pytest.mark.parametrize("cfg,lengths", SMALL, ids=[c.name for c, _ in SMALL])
+def test_small_configs(cfg, lengths):
+    w, mel, got, n_out, p_out, d_out = _run_case(cfg, np.array(lengths, np.int32))
+    assert got.shape == (cfg.batch, p_out, d_out)
+    assert p_out == O.pooled_positions(O.encoder_positions(cfg.frames), cfg.pool_step)
+    for b, ln in enumerate(lengths):
+        assert n_out[b] == O.valid_output_rows(cfg, ln)
+        ref = oracle_clip(cfg, w, mel[b], ln)
+        assert_parity(cfg, compare(cfg, got[b], ref, int(n_out[b])))
+
+
+def test_tiny_fp32_whole():
+    """The 2 s, 2-layer Whisper-large-width case in fp32 check mode: max-abs <= 1e-4."""
+    cfg = S.CONFIGS["tiny_fp32"]
+    lengths = S.make_lengths(cfg)
+    w, mel, got, n_out, p_out, d_out = _run_case(cfg, lengths)
+    assert (p_out, d_out) == (100, 1280) and n_out[0] == 100
+    ref = oracle_clip(cfg, w, mel[0], lengths[0])
+    m = compare(cfg, got[0], ref, 100)
+    assert m["max_abs"] <= 1e-4, m
+
+
+def test_batch_and_frame_mask_invariance():
+    """Clip b alone == clip b in a batch, and mel past a clip's length changes nothing (bit-exact)."""
+    import torch
+    cfg = _small("inv", batch=4, frames=300)
+    lengths = np.array([300, 150, 77, 299], np.int32)
+    w = S.make_weights(cfg)
+    mel = S.make_mel(cfg)
+    enc = make_encoder(cfg, to_device(cfg, w))
+    full = run_gpu(enc, cfg, mel, lengths)
+    alone = run_gpu(enc, cfg, mel[2:3], lengths[2:3])
+    np.testing.assert_array_equal(alone[0], full[2])
+    mel2 = mel.copy()
+    for b, ln in enumerate(lengths):
+        mel2[b, :, ln:] = S.round_bf16(np.full((cfg.n_mels, cfg.frames - ln), 7.0, np.float32))
+    np.testing.assert_array_equal(run_gpu(enc, cfg, mel2, lengths), full)
+    enc.close()
+
+
+def test_argument_errors():
+    import torch
+    from audio_encoder_tower_b200 import EncError
+    cfg = _small("err", n_layers=1)
+    w = to_device(cfg, S.make_weights(cfg))
+    enc = make_encoder(cfg, w)
+    mel = torch.zeros((cfg.batch, cfg.n_mels, cfg.frames), dtype=torch.bfloat16, device="cuda")
+    for bad in ([0, 5, 5], [5, cfg.frames + 1, 5], [-3, 1, 1]):
+        with pytest.raises(EncError) as ei:
+            enc.forward(mel, np.array(bad, np.int32))
+        assert ei.value.code == 1
+    big = torch.zeros((cfg.batch + 1, cfg.n_mels, cfg.frames), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(EncError):
+        enc.forward(big)
+    enc.status()
+    enc.close()
+    for kw, code in [(dict(n_heads=3), 2), (dict(d_model=200, n_heads=4), 2), (dict(pool_step=3), 2),
+                     (dict(n_mels=81), 2), (dict(ffn_dim=100), 2)]:
+        c2 = cfg.replace(**kw)
+        with pytest.raises(EncError) as ei:
+            make_encoder(c2, w)
+        assert ei.value.code == code, kw
+
+
+# ------------------------------------------------------------- full sizes
+FULL = [("medium_pool", [0]), ("large_b16", [5]), ("large_proj_b32", [31]), ("large_ragged_b64", None)]
+
+
+@pytest.mark.parametrize("name,sample", FULL, ids=[n for n, _ in FULL])
+def test_full_size_sampled(name, sample):
+    cfg = S.CONFIGS[name]
+    lengths = S.make_lengths(cfg)
+    if sample is None:                       # the ragged sweep: its shortest and longest clip
+        sample = [int(np.argmin(lengths)), int(np.argmax(lengths))]
+    w = S.make_weights(cfg)
+    mel = S.make_mel(cfg)
+    enc = make_encoder(cfg, to_device(cfg, w))
+    got = run_gpu(enc, cfg, mel, lengths)
+    n_out, p_out, d_out = enc.output_positions(cfg.batch, lengths)
+    enc.close()
+    assert got.shape == (cfg.batch, p_out, d_out)
+    # shapes and padding masks, every clip (bit-exact)
+    for b in range(cfg.batch):
+        assert n_out[b] == O.valid_output_rows(cfg, lengths[b])
+        assert np.all(got[b, n_out[b]:] == 0.0)
+        assert np.all(np.isfinite(got[b]))
+    for b in sample:
+        ref = oracle_clip(cfg, w, mel[b], lengths[b])
+        assert_parity(cfg, compare(cfg, got[b], ref, int(n_out[b])))
