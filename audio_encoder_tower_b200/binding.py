@@ -20,7 +20,11 @@ ENC_OK, ENC_ERR_INVALID_ARG, ENC_ERR_UNSUPPORTED, ENC_ERR_OOM, ENC_ERR_CUDA, ENC
 ENC_DTYPE_BF16, ENC_DTYPE_FP32 = 0, 1
 
 EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status", "enc_destroy",
-            "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16"]
+            "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
+            "enc_profile_enable", "enc_profile_collect", "enc_launch_count"]
+
+KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
+                  "zero"]
 
 
 class EncError(RuntimeError):
@@ -41,6 +45,10 @@ _VP = ctypes.c_void_p
 _VPP = ctypes.POINTER(ctypes.c_void_p)
 LAYER_FIELDS = ["ln1_g", "ln1_b", "q_w", "q_b", "k_w", "k_b", "v_w", "v_b", "o_w", "o_b", "ln2_g", "ln2_b",
                 "fc1_w", "fc1_b", "fc2_w", "fc2_b"]
+
+
+class EncKernelTimes(ctypes.Structure):
+    _fields_ = [("ms", ctypes.c_double * 13), ("flops", ctypes.c_double * 13), ("launches", ctypes.c_int64 * 13)]
 
 
 class EncWeights(ctypes.Structure):
@@ -81,6 +89,12 @@ def load_library(path: str = LIB_PATH):
     lib.enc_linear_bf16.restype = ctypes.c_int
     lib.enc_attention_bf16.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP]
     lib.enc_attention_bf16.restype = ctypes.c_int
+    lib.enc_profile_enable.argtypes = [_VP, ctypes.c_int32]
+    lib.enc_profile_enable.restype = ctypes.c_int
+    lib.enc_profile_collect.argtypes = [_VP, ctypes.POINTER(EncKernelTimes)]
+    lib.enc_profile_collect.restype = ctypes.c_int
+    lib.enc_launch_count.argtypes = [_VP]
+    lib.enc_launch_count.restype = ctypes.c_int64
     _LIB = lib
     return lib
 
@@ -171,6 +185,20 @@ class Encoder:
     def status(self, stream=None):
         """Synchronise `stream` and raise if a device-side check or wait failed."""
         _check(self.lib.enc_get_status(self.handle, _stream_handle(stream)), "enc_get_status")
+
+    def profile(self, enable: bool):
+        """Bracket every kernel of the following forwards with CUDA events."""
+        _check(self.lib.enc_profile_enable(self.handle, 1 if enable else 0), "enc_profile_enable")
+
+    def collect_profile(self) -> dict:
+        """{class: (ms, flops, launches)} summed since the last collect (waits for the events)."""
+        t = EncKernelTimes()
+        _check(self.lib.enc_profile_collect(self.handle, ctypes.byref(t)), "enc_profile_collect")
+        return {k: (t.ms[i], t.flops[i], int(t.launches[i])) for i, k in enumerate(KERNEL_CLASSES)
+                if t.launches[i]}
+
+    def launch_count(self) -> int:
+        return int(self.lib.enc_launch_count(self.handle))
 
     def device_bytes(self) -> int:
         return int(self.lib.enc_device_bytes(self.handle))

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "../../include/enc.h"
+#include "../../include/enc_profile.h"
 #include "common.cuh"
 #include "internal.h"
 
@@ -56,6 +57,12 @@ struct enc_handle {
   CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1;
   CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
   std::vector<LayerMaps> lmaps;
+  // profiling
+  bool profile = false;
+  int64_t launches = 0;
+  struct Rec { int cls; cudaEvent_t a, b; double flops; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> event_pool;
 };
 
 namespace {
@@ -104,6 +111,10 @@ void free_all(enc_handle* h) {
   h->h_meta = nullptr;
   if (h->meta_free) cudaEventDestroy(h->meta_free);
   h->meta_free = nullptr;
+  for (auto& r : h->recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+  h->recs.clear();
+  for (cudaEvent_t e : h->event_pool) cudaEventDestroy(e);
+  h->event_pool.clear();
 }
 
 enc_status validate_config(const enc_config* c) {
@@ -261,16 +272,55 @@ EpiParams epi_base(int mode) {
   return e;
 }
 
+cudaEvent_t pooled_event(enc_handle* h) {
+  if (!h->event_pool.empty()) {
+    cudaEvent_t e = h->event_pool.back();
+    h->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Enqueue one kernel: bracket it with events when profiling, count it.
+template <typename F>
+cudaError_t run(enc_handle* h, cudaStream_t s, int cls, double flops, F&& launch) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (h->profile) {
+    a = pooled_event(h);
+    b = pooled_event(h);
+    if (a) cudaEventRecord(a, s);
+  }
+  cudaError_t e = launch();
+  ++h->launches;
+  if (h->profile && a && b) {
+    cudaEventRecord(b, s);
+    h->recs.push_back({cls, a, b, flops});
+  }
+  return e;
+}
+
+#define ENC_RUN(cls, flops, expr) ENC_TRY(run(h, s, (cls), (flops), [&]() { return (expr); }))
+
 // ------------------------------------------------------------- forward (bf16)
-enc_status forward_bf16(enc_handle* h, const void* mel, int B, void* out, int R, int R_out, int max_n,
-                        cudaStream_t s) {
+// Sizes of one batch: packed rows, pooled/packed output rows, longest clip,
+// and sum of n_b^2 (attention work).
+struct Work {
+  int B, R, R_out, max_n;
+  double sum_n2;
+};
+
+enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& wk, cudaStream_t s) {
   const enc_config& c = h->cfg;
-  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
+  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels, B = wk.B, R = wk.R;
+  const double Rd = (double)R * d;
   const int* cu = h->meta;
   const int* cu_out = h->meta + (B + 1);
   const int* len = h->meta + 2 * (B + 1);
   bf16* melT_data = reinterpret_cast<bf16*>(h->melT) + M;
-  ENC_TRY(launch_mel_stage<bf16>(reinterpret_cast<const bf16*>(mel), len, melT_data, B, M, h->T, h->Tp, s));
+  ENC_RUN(ENC_K_MEL, 0.0,
+          launch_mel_stage<bf16>(reinterpret_cast<const bf16*>(mel), len, melT_data, B, M, h->T, h->Tp, s));
 
   GemmTcParams g;
   memset(&g, 0, sizeof(g));
@@ -279,118 +329,132 @@ enc_status forward_bf16(enc_handle* h, const void* mel, int B, void* out, int R,
   g.M = B * h->Tp; g.N = d; g.a_mode = A_CONV1; g.kb_seg = h->mpad / 64; g.num_kb = 3 * g.kb_seg;
   g.epi = epi_base(EPI_CONV1);
   g.epi.bias = h->conv1_b; g.epi.out = h->y1; g.epi.ldo = d; g.epi.T = h->T; g.epi.Tp = h->Tp;
-  ENC_TRY(launch_gemm_tc(h->m_conv1_a, h->m_conv1_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_CONV1, 2.0 * 2 * Rd * 3 * M, launch_gemm_tc(h->m_conv1_a, h->m_conv1_w, g, h->sm_count, s));
   // conv2 (+ GELU + position table) -> packed residual stream
   g.M = B * h->P1; g.N = d; g.a_mode = A_CONV2; g.kb_seg = d / 64; g.num_kb = 3 * g.kb_seg;
   g.epi = epi_base(EPI_CONV2);
   g.epi.bias = h->conv2_b; g.epi.resid = h->x; g.epi.ldo = d; g.epi.pe = h->pe; g.epi.cu = cu; g.epi.P1 = h->P1;
-  ENC_TRY(launch_gemm_tc(h->m_conv2_a, h->m_conv2_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_CONV2, 2.0 * Rd * 3 * d, launch_gemm_tc(h->m_conv2_a, h->m_conv2_w, g, h->sm_count, s));
 
+  bf16* a = reinterpret_cast<bf16*>(h->a);
   for (int l = 0; l < c.n_layers; ++l) {
     const LayerMaps& lm = h->lmaps[l];
-    ENC_TRY(launch_layernorm<bf16>(h->x, h->ln1_g[l], h->ln1_b[l], reinterpret_cast<bf16*>(h->a), R, d, c.ln_eps, s));
+    ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<bf16>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
     g.M = R; g.a_mode = A_PLAIN; g.kb_seg = 0;
     g.N = 3 * d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_STORE);
     g.epi.bias = h->qkv_b[l]; g.epi.out = h->qkv; g.epi.ldo = 3 * d;
-    ENC_TRY(launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s));
-    ENC_TRY(launch_attention_bf16(reinterpret_cast<const bf16*>(h->qkv), reinterpret_cast<bf16*>(h->o), cu, B, max_n,
-                                  d, c.n_heads, s));
+    ENC_RUN(ENC_K_QKV, 6.0 * Rd * d, launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s));
+    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d,
+            launch_attention_bf16(reinterpret_cast<const bf16*>(h->qkv), reinterpret_cast<bf16*>(h->o), cu, B,
+                                  wk.max_n, d, c.n_heads, s));
     g.N = d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->o_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
-    ENC_TRY(launch_gemm_tc(h->m_o, lm.o, g, h->sm_count, s));
-    ENC_TRY(launch_layernorm<bf16>(h->x, h->ln2_g[l], h->ln2_b[l], reinterpret_cast<bf16*>(h->a), R, d, c.ln_eps, s));
+    ENC_RUN(ENC_K_OUT, 2.0 * Rd * d, launch_gemm_tc(h->m_o, lm.o, g, h->sm_count, s));
+    ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<bf16>(h->x, h->ln2_g[l], h->ln2_b[l], a, R, d, c.ln_eps, s));
     g.N = F; g.num_kb = d / 64;
     g.epi = epi_base(EPI_STORE);
     g.epi.gelu = 1; g.epi.bias = h->fc1_b[l]; g.epi.out = h->f; g.epi.ldo = F;
-    ENC_TRY(launch_gemm_tc(h->m_a, lm.fc1, g, h->sm_count, s));
+    ENC_RUN(ENC_K_FC1, 2.0 * Rd * F, launch_gemm_tc(h->m_a, lm.fc1, g, h->sm_count, s));
     g.N = d; g.num_kb = F / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->fc2_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
-    ENC_TRY(launch_gemm_tc(h->m_f, lm.fc2, g, h->sm_count, s));
+    ENC_RUN(ENC_K_FC2, 2.0 * Rd * F, launch_gemm_tc(h->m_f, lm.fc2, g, h->sm_count, s));
   }
 
   if (!c.proj_hidden) {
-    ENC_TRY(launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(out), B,
+    ENC_RUN(ENC_K_FINAL, 0.0,
+            launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(out), B,
                                   h->p_out, d, c.pool_step, 0, c.ln_eps, s));
     return ENC_OK;
   }
   const int ph = c.proj_hidden, po = c.proj_out;
-  ENC_TRY(launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(h->e), B,
+  const double Ro = wk.R_out;
+  ENC_RUN(ENC_K_FINAL, 0.0,
+          launch_final_ln<bf16>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<bf16*>(h->e), B,
                                 h->p_out, d, c.pool_step, 1, c.ln_eps, s));
-  g.M = R_out; g.a_mode = A_PLAIN; g.kb_seg = 0;
+  g.M = wk.R_out; g.a_mode = A_PLAIN; g.kb_seg = 0;
   g.N = ph; g.num_kb = d / 64;
   g.epi = epi_base(EPI_STORE);
   g.epi.gelu = 1; g.epi.bias = h->proj1_b; g.epi.out = h->p1; g.epi.ldo = ph;
-  ENC_TRY(launch_gemm_tc(h->m_e, h->m_proj1_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_PROJ1, 2.0 * Ro * d * ph, launch_gemm_tc(h->m_e, h->m_proj1_w, g, h->sm_count, s));
   g.N = po; g.num_kb = ph / 64;
   g.epi = epi_base(EPI_SCATTER);
   g.epi.bias = h->proj2_b; g.epi.out = out; g.epi.ldo = po; g.epi.cu = cu_out; g.epi.B = B; g.epi.p_out = h->p_out;
-  ENC_TRY(launch_gemm_tc(h->m_p1, h->m_proj2_w, g, h->sm_count, s));
-  ENC_TRY(launch_zero_tail_rows<bf16>(reinterpret_cast<bf16*>(out), cu_out, B, h->p_out, po, s));
+  ENC_RUN(ENC_K_PROJ2, 2.0 * Ro * ph * po, launch_gemm_tc(h->m_p1, h->m_proj2_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_ZERO, 0.0, launch_zero_tail_rows<bf16>(reinterpret_cast<bf16*>(out), cu_out, B, h->p_out, po, s));
   return ENC_OK;
 }
 
 // -------------------------------------------------------- forward (fp32 check)
-enc_status forward_f32(enc_handle* h, const void* mel, int B, void* out, int R, int R_out, int max_n,
-                       cudaStream_t s) {
+enc_status forward_f32(enc_handle* h, const void* mel, void* out, const Work& wk, cudaStream_t s) {
   const enc_config& c = h->cfg;
-  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
+  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels, B = wk.B, R = wk.R;
+  const double Rd = (double)R * d;
   const int* cu = h->meta;
   const int* cu_out = h->meta + (B + 1);
   const int* len = h->meta + 2 * (B + 1);
   float* melT = reinterpret_cast<float*>(h->melT);
   float* y1 = reinterpret_cast<float*>(h->y1);
-  ENC_TRY(launch_mel_stage<float>(reinterpret_cast<const float*>(mel), len, melT + M, B, M, h->T, h->Tp, s));
+  ENC_RUN(ENC_K_MEL, 0.0,
+          launch_mel_stage<float>(reinterpret_cast<const float*>(mel), len, melT + M, B, M, h->T, h->Tp, s));
 
   EpiParams e = epi_base(EPI_CONV1);
   e.bias = h->conv1_b; e.out = y1; e.ldo = d; e.T = h->T; e.Tp = h->Tp;
   // conv1 row r reads mel rows r-1, r, r+1: A starts at the guard row, rows overlap (lda = M)
-  ENC_TRY(launch_sgemm(melT, M, reinterpret_cast<const float*>(h->conv1_w), 3 * M, B * h->Tp, d, 3 * M, e, s));
+  ENC_RUN(ENC_K_CONV1, 2.0 * 2 * Rd * 3 * M,
+          launch_sgemm(melT, M, reinterpret_cast<const float*>(h->conv1_w), 3 * M, B * h->Tp, d, 3 * M, e, s));
   e = epi_base(EPI_CONV2);
   e.bias = h->conv2_b; e.resid = h->x; e.ldo = d; e.pe = h->pe; e.cu = cu; e.P1 = h->P1;
   // conv2 row j reads conv1 rows 2j, 2j+1, 2j+2 (padded time): lda = 2d, K = 3d
-  ENC_TRY(launch_sgemm(y1, 2 * d, reinterpret_cast<const float*>(h->conv2_w), 3 * d, B * h->P1, d, 3 * d, e, s));
+  ENC_RUN(ENC_K_CONV2, 2.0 * Rd * 3 * d,
+          launch_sgemm(y1, 2 * d, reinterpret_cast<const float*>(h->conv2_w), 3 * d, B * h->P1, d, 3 * d, e, s));
 
   float* a = reinterpret_cast<float*>(h->a);
   float* qkv = reinterpret_cast<float*>(h->qkv);
   float* o = reinterpret_cast<float*>(h->o);
   float* f = reinterpret_cast<float*>(h->f);
   for (int l = 0; l < c.n_layers; ++l) {
-    ENC_TRY(launch_layernorm<float>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
+    ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<float>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
     e = epi_base(EPI_STORE);
     e.bias = h->qkv_b[l]; e.out = qkv; e.ldo = 3 * d;
-    ENC_TRY(launch_sgemm(a, d, reinterpret_cast<const float*>(h->qkv_w[l]), d, R, 3 * d, d, e, s));
-    ENC_TRY(launch_attention_f32(qkv, o, cu, B, max_n, d, c.n_heads, s));
+    ENC_RUN(ENC_K_QKV, 6.0 * Rd * d,
+            launch_sgemm(a, d, reinterpret_cast<const float*>(h->qkv_w[l]), d, R, 3 * d, d, e, s));
+    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d, launch_attention_f32(qkv, o, cu, B, wk.max_n, d, c.n_heads, s));
     e = epi_base(EPI_RESIDUAL);
     e.bias = h->o_b[l]; e.resid = h->x; e.ldo = d;
-    ENC_TRY(launch_sgemm(o, d, reinterpret_cast<const float*>(h->o_w[l]), d, R, d, d, e, s));
-    ENC_TRY(launch_layernorm<float>(h->x, h->ln2_g[l], h->ln2_b[l], a, R, d, c.ln_eps, s));
+    ENC_RUN(ENC_K_OUT, 2.0 * Rd * d, launch_sgemm(o, d, reinterpret_cast<const float*>(h->o_w[l]), d, R, d, d, e, s));
+    ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<float>(h->x, h->ln2_g[l], h->ln2_b[l], a, R, d, c.ln_eps, s));
     e = epi_base(EPI_STORE);
     e.gelu = 1; e.bias = h->fc1_b[l]; e.out = f; e.ldo = F;
-    ENC_TRY(launch_sgemm(a, d, reinterpret_cast<const float*>(h->fc1_w[l]), d, R, F, d, e, s));
+    ENC_RUN(ENC_K_FC1, 2.0 * Rd * F, launch_sgemm(a, d, reinterpret_cast<const float*>(h->fc1_w[l]), d, R, F, d, e, s));
     e = epi_base(EPI_RESIDUAL);
     e.bias = h->fc2_b[l]; e.resid = h->x; e.ldo = d;
-    ENC_TRY(launch_sgemm(f, F, reinterpret_cast<const float*>(h->fc2_w[l]), F, R, d, F, e, s));
+    ENC_RUN(ENC_K_FC2, 2.0 * Rd * F, launch_sgemm(f, F, reinterpret_cast<const float*>(h->fc2_w[l]), F, R, d, F, e, s));
   }
   if (!c.proj_hidden) {
-    ENC_TRY(launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<float*>(out), B,
+    ENC_RUN(ENC_K_FINAL, 0.0,
+            launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, reinterpret_cast<float*>(out), B,
                                    h->p_out, d, c.pool_step, 0, c.ln_eps, s));
     return ENC_OK;
   }
   const int ph = c.proj_hidden, po = c.proj_out;
+  const double Ro = wk.R_out;
   float* ev = reinterpret_cast<float*>(h->e);
   float* p1 = reinterpret_cast<float*>(h->p1);
-  ENC_TRY(launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, ev, B, h->p_out, d, c.pool_step, 1,
+  ENC_RUN(ENC_K_FINAL, 0.0,
+          launch_final_ln<float>(h->x, h->lnpost_g, h->lnpost_b, cu, cu_out, ev, B, h->p_out, d, c.pool_step, 1,
                                  c.ln_eps, s));
   e = epi_base(EPI_STORE);
   e.gelu = 1; e.bias = h->proj1_b; e.out = p1; e.ldo = ph;
-  ENC_TRY(launch_sgemm(ev, d, reinterpret_cast<const float*>(h->proj1_w), d, R_out, ph, d, e, s));
+  ENC_RUN(ENC_K_PROJ1, 2.0 * Ro * d * ph,
+          launch_sgemm(ev, d, reinterpret_cast<const float*>(h->proj1_w), d, wk.R_out, ph, d, e, s));
   e = epi_base(EPI_SCATTER);
   e.bias = h->proj2_b; e.out = out; e.ldo = po; e.cu = cu_out; e.B = B; e.p_out = h->p_out;
-  ENC_TRY(launch_sgemm(p1, ph, reinterpret_cast<const float*>(h->proj2_w), ph, R_out, po, ph, e, s));
-  ENC_TRY(launch_zero_tail_rows<float>(reinterpret_cast<float*>(out), cu_out, B, h->p_out, po, s));
+  ENC_RUN(ENC_K_PROJ2, 2.0 * Ro * ph * po,
+          launch_sgemm(p1, ph, reinterpret_cast<const float*>(h->proj2_w), ph, wk.R_out, po, ph, e, s));
+  ENC_RUN(ENC_K_ZERO, 0.0, launch_zero_tail_rows<float>(reinterpret_cast<float*>(out), cu_out, B, h->p_out, po, s));
   return ENC_OK;
 }
 
@@ -472,6 +536,7 @@ enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, i
   // per-clip counts (host): n_b = ceil(len_b / 2) positions, packed offsets
   std::vector<int> len(B), cu(B + 1), cu_out(B + 1);
   int max_n = 0;
+  double sum_n2 = 0.0;
   cu[0] = cu_out[0] = 0;
   for (int b = 0; b < B; ++b) {
     len[b] = lengths ? lengths[b] : h->T;
@@ -480,6 +545,7 @@ enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, i
     cu[b + 1] = cu[b] + n;
     cu_out[b + 1] = cu_out[b] + valid_out(h, n);
     if (n > max_n) max_n = n;
+    sum_n2 += (double)n * n;
   }
   if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
   // the pinned staging buffer may still feed the previous forward's upload
@@ -491,9 +557,8 @@ enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, i
   ENC_TRY(cudaMemcpyAsync(h->meta, hm, (size_t)(3 * B + 2) * 4, cudaMemcpyHostToDevice, stream));
   ENC_TRY(cudaEventRecord(h->meta_free, stream));
   h->meta_pending = true;
-  const int R = cu[B], R_out = cu_out[B];
-  return h->bf16 ? forward_bf16(h, mel, B, out, R, R_out, max_n, stream)
-                 : forward_f32(h, mel, B, out, R, R_out, max_n, stream);
+  const Work wk{B, cu[B], cu_out[B], max_n, sum_n2};
+  return h->bf16 ? forward_bf16(h, mel, out, wk, stream) : forward_f32(h, mel, out, wk, stream);
 }
 
 enc_status enc_get_status(enc_handle* h, cudaStream_t stream) {
@@ -518,5 +583,37 @@ void enc_destroy(enc_handle* h) {
 }
 
 size_t enc_device_bytes(const enc_handle* h) { return h ? h->bytes : 0; }
+
+enc_status enc_profile_enable(enc_handle* h, int32_t enable) {
+  if (!h) return ENC_ERR_INVALID_ARG;
+  h->profile = enable != 0;
+  return ENC_OK;
+}
+
+enc_status enc_profile_collect(enc_handle* h, enc_kernel_times* out) {
+  if (!h || !out) return ENC_ERR_INVALID_ARG;
+  memset(out, 0, sizeof(*out));
+  if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
+  enc_status st = ENC_OK;
+  for (const auto& r : h->recs) {
+    float ms = 0.f;
+    if (st == ENC_OK) {
+      cudaError_t e = cudaEventSynchronize(r.b);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+      if (e != cudaSuccess) st = cuda_status(e);
+    }
+    if (r.cls >= 0 && r.cls < ENC_K_COUNT) {
+      out->ms[r.cls] += ms;
+      out->flops[r.cls] += r.flops;
+      out->launches[r.cls] += 1;
+    }
+    h->event_pool.push_back(r.a);
+    h->event_pool.push_back(r.b);
+  }
+  h->recs.clear();
+  return st;
+}
+
+int64_t enc_launch_count(const enc_handle* h) { return h ? h->launches : 0; }
 
 }  // extern "C"

@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Throughput of the Whisper-style audio encoder tower forward pass on B200.
+
+Default workload: the Whisper-large encoder (32 layers, d_model 1280, 20 heads
+x 64, FFN 5120, 128 mel bins x 3000 frames = 30 s per clip -> 1500 positions),
+batch 16 per GPU, bf16 operands with fp32 accumulation, synthetic seeded inputs
+and random weights of that architecture.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one enc_forward over a batch of 16 clips. Multi-GPU (torchrun, one
+process per GPU) runs independent replicas, each with its own batch of 16
+(weak scaling, no collective on the data path); the time is the max over ranks.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic as S  # noqa: E402
+
+METRIC = "audio-sec/s and TFLOP/s (% of BF16 peak), Whisper-large encoder, B=16, bf16, 1 B200"
+UNIT = "audio-s/s"
+FRAMES_PER_SECOND = 100.0          # 16 kHz audio, hop 160
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_CLASSES = ("conv1", "conv2", "qkv", "out", "fc1", "fc2", "proj1", "proj2")
+
+
+# ----------------------------------------------------------------- workload
+def workload_flops(cfg, lengths, layers=None) -> float:
+    """Algorithmic FLOPs (multiply-add = 2) over the valid positions of each clip."""
+    d, m, f = cfg.d_model, cfg.n_mels, cfg.ffn_dim
+    L = cfg.n_layers if layers is None else layers
+    total = 0.0
+    for ln in lengths:
+        n = (int(ln) + 1) // 2
+        total += 2.0 * (2 * n) * d * 3 * m + 2.0 * n * d * 3 * d
+        total += L * (6.0 * n * d * d + 4.0 * n * n * d + 2.0 * n * d * d + 4.0 * n * d * f)
+        if cfg.proj_hidden:
+            no = n // cfg.pool_step if cfg.pool_step > 1 else n
+            total += 2.0 * no * (d * cfg.proj_hidden + cfg.proj_hidden * cfg.proj_out)
+    return total
+
+
+def workload_desc(cfg, n_gpus):
+    return {
+        "workload": (f"{cfg.name}: Whisper-style encoder {cfg.n_layers}L d{cfg.d_model} {cfg.n_heads}x64 heads "
+                     f"FFN{cfg.ffn_dim}, {cfg.n_mels} mel x {cfg.frames} frames, B={cfg.batch} per GPU"
+                     + (f", pool {cfg.pool_step}" if cfg.pool_step > 1 else "")
+                     + (f", projector {cfg.d_model}->{cfg.proj_hidden}->{cfg.proj_out}" if cfg.proj_hidden else "")
+                     + (f", lengths U[{cfg.ragged[0]},{cfg.ragged[1]}] frames" if cfg.ragged else "")),
+        "global_batch": cfg.batch * n_gpus,
+        "frames": cfg.frames,
+        "positions": cfg.positions,
+        "parallelism": f"replicas x{n_gpus} (batch sharded, no collective)",
+        "l2": "per-step working set >> 126 MB L2 (weights 1.27 GB bf16 + activations), no explicit flush",
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------- oracle legs
+def oracle_sample(cfg, w, mel_clip, length, layers):
+    """Time the oracle on one clip: conv stem + `layers` blocks + final LN."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.encode_clip(cfg, w, mel_clip, int(length), layers=layers)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, layers=8):
+    """The oracle on the host cores, on a bounded sample of the same workload."""
+    lengths = S.make_lengths(cfg)
+    w = S.make_weights(cfg, layers=list(range(layers)))
+    mel = S.mel_clip(cfg, 0)
+    secs = oracle_sample(cfg, w, mel, lengths[0], layers)
+    sample_flops = workload_flops(cfg, lengths[:1], layers)
+    flops_per_audio_s = workload_flops(cfg, lengths) / (float(np.sum(lengths)) / FRAMES_PER_SECOND)
+    return {"value": sample_flops / secs / flops_per_audio_s, "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": (f"1 clip ({lengths[0]} frames), conv stem + {layers} of {cfg.n_layers} blocks + final LN, "
+                       f"float64 numpy/BLAS, {secs:.2f} s; audio-s/s at the full workload's FLOPs per audio second"),
+            "seconds": secs}
+
+
+def run_reference(args, cfg):
+    """--impl reference: the oracle (float64, host cores) timed on this workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    layers = 1
+    lengths = S.make_lengths(cfg)
+    w = S.make_weights(cfg, layers=list(range(layers)))
+    mel = S.mel_clip(cfg, 0)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, w, mel, lengths[0], layers)
+    times = [oracle_sample(cfg, w, mel, lengths[0], layers) for _ in range(args.steps)]
+    tot = sum(times)
+    sample_flops = workload_flops(cfg, lengths[:1], layers)
+    flops_per_audio_s = workload_flops(cfg, lengths) / (float(np.sum(lengths)) / FRAMES_PER_SECOND)
+    value = sample_flops * args.steps / tot / flops_per_audio_s
+    sample = (f"each step: 1 clip ({lengths[0]} frames), conv stem + {layers} of {cfg.n_layers} blocks + final LN, "
+              f"float64 numpy/BLAS; audio-s/s at the full workload's FLOPs per audio second")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.rows = []
+        ident = str(device_index)
+        try:
+            import torch
+            u = getattr(torch.cuda.get_device_properties(device_index), "uuid", None)
+            if u is not None:
+                ident = "GPU-" + str(u)
+        except Exception:
+            pass
+        self.ident = ident
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 8:
+                self.rows.append(parts)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        pw = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows), "power_w_max": max(pw) if pw else None}
+
+
+def gemm_traffic_record():
+    """DRAM traffic of the GEMM kernel from a committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for fn in ("gemm_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "audio_encoder_tower_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return rec if rec.get("source_sha256") == h.hexdigest() else None
+
+
+# ---------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="large_b16", choices=S.CONFIG_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = S.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import torch.distributed as dist
+    from audio_encoder_tower_b200 import Encoder
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- synthetic inputs and weights (per rank: own clips, same weights)
+    w_np = S.make_weights(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    w_dev = {k: torch.from_numpy(v).to(device=dev, dtype=dt) for k, v in w_np.items()}
+    del w_np
+    rcfg = cfg.replace(seed=cfg.seed + 1000 * rank) if rank else cfg
+    lengths = S.make_lengths(rcfg)
+    mel_np = S.make_mel(rcfg)
+    enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
+                  ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=cfg.batch, dtype=cfg.dtype,
+                  pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out, weights=w_dev)
+    del w_dev
+    torch.cuda.empty_cache()
+    mel = torch.from_numpy(mel_np).to(device=dev, dtype=dt)
+    _, p_out, d_out = enc.output_positions(cfg.batch, lengths)
+    out = torch.empty((cfg.batch, p_out, d_out), dtype=dt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    audio_s = float(np.sum(lengths)) / FRAMES_PER_SECOND
+    flops = workload_flops(cfg, lengths)
+
+    # ---- device-resident timing (inputs in HBM when the region starts)
+    for _ in range(args.warmup):
+        enc.forward(mel, lengths, out, stream)
+    enc.status(stream)
+    enc.profile(True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = enc.launch_count()
+    e0.record(stream)
+    for _ in range(args.steps):
+        enc.forward(mel, lengths, out, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = enc.launch_count() - n0
+    clocks.stop()
+    enc.profile(False)
+    prof = enc.collect_profile()
+    enc.status(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # ---- end to end through the public call with host buffers
+    mel_host = torch.from_numpy(mel_np).to(dtype=dt).pin_memory()
+    out_host = torch.empty(out.shape, dtype=dt).pin_memory()
+    mel_in = torch.empty_like(mel)
+
+    def e2e_step():
+        mel_in.copy_(mel_host, non_blocking=True)
+        enc.forward(mel_in, lengths, out, stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    enc.status(stream)
+    if not np.all(np.isfinite(out_host[0, :10].float().numpy())):
+        raise RuntimeError("non-finite encoder output")
+
+    # ---- roofline of the dominant kernel (the tcgen05 GEMM, every GEMM launch of the region)
+    peaks, peak_src = load_peaks()
+    g_ms = sum(prof[k][0] for k in GEMM_CLASSES if k in prof)
+    g_fl = sum(prof[k][1] for k in GEMM_CLASSES if k in prof)
+    g_n = sum(prof[k][2] for k in GEMM_CLASSES if k in prof)
+    step_ms_prof = sum(v[0] for v in prof.values())
+    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ach = (g_fl / g_n) / (g_ms / g_n) / 1e9 if g_n else 0.0
+    traffic = gemm_traffic_record()
+    roofline = {"kernel": "gemm_tc_kernel (tcgen05, all GEMM launches of the timed region)",
+                "bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "frac_of_burst_peak": ach / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+                "traffic": (traffic["bytes_per_launch"] if traffic else None),
+                "share_of_step": g_ms / step_ms_prof if step_ms_prof else None,
+                "launches": g_n, "flops_per_launch": g_fl / g_n if g_n else None}
+    kernels = {k: {"ms_per_step": v[0] / args.steps, "tflops": (v[1] / v[0] / 1e9 if v[0] and v[1] else None),
+                   "share": v[0] / step_ms_prof} for k, v in prof.items()}
+
+    tflops = flops / ms / 1e9
+    line = {"metric": METRIC, "value": world * audio_s / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; random weights)",
+            "config": workload_desc(cfg, world),
+            "tflops": world * tflops,
+            "frac_bf16_peak": tflops / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+            "frac_bf16_peak_sustained": tflops / peak_tf,
+            "peaks": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+            "roofline": roofline,
+            "kernels": kernels,
+            "e2e": {"value": world * audio_s / (ms_e2e / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(mel_host.numel() * mel_host.element_size()),
+                    "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+                    "ms_per_step": ms_e2e, "api": "enc_forward (C ABI) + pinned host copies on the same stream"},
+            "gpu_launches": int(launches),
+            "clocks": clocks.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    enc.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
