@@ -21,7 +21,7 @@ ENC_DTYPE_BF16, ENC_DTYPE_FP32 = 0, 1
 
 EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status", "enc_destroy",
             "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
-            "enc_profile_enable", "enc_profile_collect", "enc_launch_count"]
+            "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch"]
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -95,6 +95,8 @@ def load_library(path: str = LIB_PATH):
     lib.enc_profile_collect.restype = ctypes.c_int
     lib.enc_launch_count.argtypes = [_VP]
     lib.enc_launch_count.restype = ctypes.c_int64
+    lib.enc_forward_static_scratch.argtypes = [_VP, _VP, i32p, ctypes.c_int32, _VP, _VP]
+    lib.enc_forward_static_scratch.restype = ctypes.c_int
     _LIB = lib
     return lib
 
@@ -180,6 +182,26 @@ class Encoder:
             lp = self._len.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
         _check(self.lib.enc_forward(self.handle, _ptr(mel), lp, B, _ptr(out), _stream_handle(stream)),
                "enc_forward")
+        return out
+
+    def forward_static_scratch(self, mel, lengths=None, out=None, stream=None):
+        """enc_forward_static_scratch: the same forward with its workspace in the
+        library's fixed 64 MiB static device array (no device allocation in the call).
+
+        `out` must be given by callers that cannot allocate; when omitted it is
+        allocated here with torch for convenience.
+        """
+        import torch
+        B = int(mel.shape[0])
+        if out is None:
+            _, p_out, d_out = self.output_positions(B, lengths)
+            out = torch.empty((B, p_out, d_out), dtype=mel.dtype, device=mel.device)
+        lp = None
+        if lengths is not None:
+            self._len = np.ascontiguousarray(lengths, dtype=np.int32)
+            lp = self._len.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        _check(self.lib.enc_forward_static_scratch(self.handle, _ptr(mel), lp, B, _ptr(out),
+                                                   _stream_handle(stream)), "enc_forward_static_scratch")
         return out
 
     def status(self, stream=None):

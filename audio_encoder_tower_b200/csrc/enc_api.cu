@@ -617,3 +617,134 @@ enc_status enc_profile_collect(enc_handle* h, enc_kernel_times* out) {
 int64_t enc_launch_count(const enc_handle* h) { return h ? h->launches : 0; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// enc_forward_static_scratch: the forward pass with its workspace in a fixed
+// static device array instead of handle-owned memory, so that the call itself
+// needs no device allocation. Reuses the launch sequence above unchanged.
+// ---------------------------------------------------------------------------
+#define ENC_STATIC_SCRATCH_BYTES (64ull << 20)
+
+// Reserved by the CUDA runtime on every device that loads this library, until exit.
+static __device__ __align__(256) unsigned char enc_static_scratch[ENC_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+void* g_static_scratch_base[64] = {};   // device address of enc_static_scratch, per device ordinal
+
+// Set-up, once per device, with that device current: the array's name is only a
+// host-side stand-in, so ask the runtime for its device address.
+enc_status static_scratch_base(int dev, unsigned char** base) {
+  if (dev < 0 || dev >= 64) return ENC_ERR_UNSUPPORTED;
+  if (!g_static_scratch_base[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, enc_static_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
+      return ENC_ERR_CUDA;
+    }
+    g_static_scratch_base[dev] = p;
+  }
+  *base = reinterpret_cast<unsigned char*>(g_static_scratch_base[dev]);
+  return ENC_OK;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel, const int32_t* lengths, int32_t B,
+                                                 void* out, cudaStream_t stream) {
+  if (!h || !mel || !out || B < 1 || B > h->cfg.max_batch) return ENC_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(mel) | reinterpret_cast<uintptr_t>(out)) & 15u) return ENC_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b) {
+    const int len = lengths ? lengths[b] : h->T;
+    if (len < 1 || len > h->T) return ENC_ERR_INVALID_ARG;
+  }
+  const enc_config& c = h->cfg;
+  const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
+  if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
+  unsigned char* base = nullptr;
+  enc_status st = static_scratch_base(h->device, &base);
+  if (st != ENC_OK) return st;
+
+  // per-clip counts, written straight into the handle's pinned staging buffer
+  if (h->meta_pending) ENC_TRY(cudaEventSynchronize(h->meta_free));
+  int* hcu = h->h_meta;
+  int* hcu_out = hcu + (B + 1);
+  int* hlen = hcu + 2 * (B + 1);
+  int max_n = 0;
+  double sum_n2 = 0.0;
+  hcu[0] = hcu_out[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    hlen[b] = lengths ? lengths[b] : h->T;
+    const int n = (hlen[b] + 1) / 2;
+    hcu[b + 1] = hcu[b] + n;
+    hcu_out[b + 1] = hcu_out[b] + valid_out(h, n);
+    if (n > max_n) max_n = n;
+    sum_n2 += (double)n * n;
+  }
+  const int R = hcu[B], R_out = hcu_out[B];
+
+  // carve the workspace of this batch out of the static array
+  const size_t rows_t = (size_t)B * h->Tp;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { unsigned char* p = base + off; off += align256(bytes); return p; };
+  unsigned char* melT = take((rows_t + 2) * M * h->esz);
+  unsigned char* y1 = take((rows_t + 2) * d * h->esz);
+  unsigned char* x = take((size_t)R * d * 4);
+  unsigned char* a = take((size_t)R * d * h->esz);
+  unsigned char* qkv = take((size_t)R * 3 * d * h->esz);
+  unsigned char* o = take((size_t)R * d * h->esz);
+  unsigned char* f = take((size_t)R * F * h->esz);
+  unsigned char* e = c.proj_hidden ? take((size_t)R_out * d * h->esz) : nullptr;
+  unsigned char* p1 = c.proj_hidden ? take((size_t)R_out * c.proj_hidden * h->esz) : nullptr;
+  unsigned char* meta = take((size_t)(3 * B + 2) * 4);
+  if (off > ENC_STATIC_SCRATCH_BYTES) return ENC_ERR_INVALID_ARG;   // batch too large for the array
+
+  // the array keeps the previous call's contents: clear what is read as zero
+  // (the guard rows around the time-major mel)
+  ENC_TRY(cudaMemsetAsync(melT, 0, (size_t)M * h->esz, stream));
+  ENC_TRY(cudaMemsetAsync(melT + (rows_t + 1) * M * h->esz, 0, (size_t)M * h->esz, stream));
+
+  // point the handle at the static workspace for this call, then restore it
+  void *s_melT = h->melT, *s_y1 = h->y1, *s_a = h->a, *s_qkv = h->qkv, *s_o = h->o, *s_f = h->f, *s_e = h->e,
+       *s_p1 = h->p1;
+  float* s_x = h->x;
+  int* s_meta = h->meta;
+  const CUtensorMap s_conv1_a = h->m_conv1_a, s_conv2_a = h->m_conv2_a, s_ma = h->m_a, s_mo = h->m_o,
+                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1;
+  const bool s_profile = h->profile;
+  h->melT = melT; h->y1 = y1; h->x = reinterpret_cast<float*>(x); h->a = a; h->qkv = qkv; h->o = o; h->f = f;
+  h->e = e; h->p1 = p1; h->meta = reinterpret_cast<int*>(meta);
+  h->profile = false;   // event records would grow host-side lists
+  st = ENC_OK;
+  if (h->bf16) {
+    bool ok = map_rows(&h->m_conv1_a, melT + (size_t)M * 2, M, (long long)rows_t, 128);
+    ok = ok && make_tma_2d(&h->m_conv2_a, y1, 2 * (uint64_t)d, (uint64_t)rows_t / 2, 4 * (uint64_t)d, 64, 128);
+    ok = ok && map_rows(&h->m_a, a, d, R, 128);
+    ok = ok && map_rows(&h->m_o, o, d, R, 128);
+    ok = ok && map_rows(&h->m_f, f, F, R, 128);
+    if (c.proj_hidden) {
+      ok = ok && map_rows(&h->m_e, e, d, R_out > 0 ? R_out : 1, 128);
+      ok = ok && map_rows(&h->m_p1, p1, c.proj_hidden, R_out > 0 ? R_out : 1, 128);
+    }
+    if (!ok) st = ENC_ERR_CUDA;
+  }
+  if (st == ENC_OK) {
+    cudaError_t ce = cudaMemcpyAsync(h->meta, h->h_meta, (size_t)(3 * B + 2) * 4, cudaMemcpyHostToDevice, stream);
+    if (ce == cudaSuccess) ce = cudaEventRecord(h->meta_free, stream);
+    if (ce != cudaSuccess) st = cuda_status(ce);
+    else h->meta_pending = true;
+  }
+  if (st == ENC_OK) {
+    const Work wk{B, R, R_out, max_n, sum_n2};
+    st = h->bf16 ? forward_bf16(h, mel, out, wk, stream) : forward_f32(h, mel, out, wk, stream);
+  }
+  h->melT = s_melT; h->y1 = s_y1; h->x = s_x; h->a = s_a; h->qkv = s_qkv; h->o = s_o; h->f = s_f; h->e = s_e;
+  h->p1 = s_p1; h->meta = s_meta;
+  h->m_conv1_a = s_conv1_a; h->m_conv2_a = s_conv2_a; h->m_a = s_ma; h->m_o = s_mo; h->m_f = s_mf; h->m_e = s_me;
+  h->m_p1 = s_mp1;
+  h->profile = s_profile;
+  return st;
+}

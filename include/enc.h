@@ -166,6 +166,35 @@ ENC_API const char *enc_status_string(enc_status s);
 /* Library-owned device bytes: repacked weights and workspace (for reporting). */
 ENC_API size_t enc_device_bytes(const enc_handle *h);
 
+/*
+ * enc_forward without any device allocation, for callers that cannot call
+ * cudaMalloc once they are running -- for example a serving process whose
+ * device memory is handed out up front by its own pool allocator, where a new
+ * cudaMalloc would fail or break the pool. (The model pages have no
+ * counterpart of this call; it is a property of this library.)
+ *
+ * Same arguments, output and errors as enc_forward, with the handle's weights.
+ * The per-batch workspace (time-major mel, conv1 output, residual stream, LN,
+ * QKV, attention and FFN buffers, projector buffers, clip offsets) is carved
+ * out of one file-scope static device array of 64 MiB (67,108,864 bytes) that
+ * the CUDA runtime reserves on every device that loads this library and keeps
+ * until the process exits. The call itself allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).
+ *   - Capacity: a batch whose workspace exceeds 64 MiB returns
+ *     ENC_ERR_INVALID_ARG before anything is enqueued. One 30 s clip of the
+ *     Whisper-large encoder (about 51 MB of workspace) fits; two do not.
+ *   - Set-up: the first call on a device looks up the device address of the
+ *     array (cudaGetSymbolAddress, with that device current). Make that first
+ *     call before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     previous call's contents; the call clears what it reads as zero. Calls
+ *     whose GPU work overlaps (other streams, other handles, other threads)
+ *     race on the array: order them on one stream or synchronise between them.
+ *   - Profiling (enc_profile_enable) does not record this call's kernels.
+ */
+ENC_API enc_status enc_forward_static_scratch(enc_handle *h, const void *mel, const int32_t *lengths, int32_t B,
+                                              void *out, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
