@@ -87,7 +87,8 @@ def load_library(path: str = LIB_PATH):
     lib.enc_linear_bf16.argtypes = [_VP, _VP, _VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                     ctypes.c_int32, _VP, _VP]
     lib.enc_linear_bf16.restype = ctypes.c_int
-    lib.enc_attention_bf16.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP]
+    lib.enc_attention_bf16.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32, _VP, _VP]
     lib.enc_attention_bf16.restype = ctypes.c_int
     lib.enc_profile_enable.argtypes = [_VP, ctypes.c_int32]
     lib.enc_profile_enable.restype = ctypes.c_int
@@ -251,13 +252,14 @@ def linear_bf16(A, W, bias=None, out=None, resid=None, gelu=False, status=None, 
     return out if resid is None else resid
 
 
-def attention_bf16(qkv, cu, max_n, n_heads, out=None, stream=None):
+def attention_bf16(qkv, cu, max_n, n_heads, out=None, status=None, stream=None):
     """Packed-clip bidirectional attention: qkv [R, 3d] bf16, cu device int32 [B+1]."""
     import torch
     R = qkv.shape[0]
     d = 64 * n_heads
     if out is None:
         out = torch.empty((R, d), dtype=torch.bfloat16, device=qkv.device)
-    _check(load_library().enc_attention_bf16(_ptr(qkv), _ptr(out), _ptr(cu), int(cu.numel()) - 1, int(max_n),
-                                             int(n_heads), _stream_handle(stream)), "enc_attention_bf16")
+    _check(load_library().enc_attention_bf16(_ptr(qkv), _ptr(out), _ptr(cu), int(R), int(cu.numel()) - 1,
+                                             int(max_n), int(n_heads), _ptr(status), _stream_handle(stream)),
+           "enc_attention_bf16")
     return out

@@ -54,7 +54,7 @@ struct enc_handle {
   cudaEvent_t meta_free = nullptr;
   bool meta_pending = false;
   // tensor maps (bf16 path)
-  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1;
+  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_qkv;
   CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
   std::vector<LayerMaps> lmaps;
   // profiling
@@ -227,6 +227,11 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ENC_CHECK(dev_alloc(h, &h->e, (size_t)rows_o * d * h->esz));
     ENC_CHECK(dev_alloc(h, &h->p1, (size_t)rows_o * ph * h->esz));
   }
+  ENC_TRY(cudaMemset(h->x, 0, (size_t)rows_p * d * 4));
+  ENC_TRY(cudaMemset(h->a, 0, (size_t)rows_p * d * h->esz));
+  ENC_TRY(cudaMemset(h->qkv, 0, (size_t)rows_p * 3 * d * h->esz));
+  ENC_TRY(cudaMemset(h->o, 0, (size_t)rows_p * d * h->esz));
+  ENC_TRY(cudaMemset(h->f, 0, (size_t)rows_p * F * h->esz));
   ENC_CHECK(dev_alloc(h, &h->meta, (size_t)(3 * Bm + 2) * 4));
   ENC_CHECK(dev_alloc(h, &h->status, 4));
   ENC_TRY(cudaMemset(h->status, 0, 4));
@@ -244,6 +249,7 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ok = ok && map_rows(&h->m_a, h->a, d, rows_p, 128);
     ok = ok && map_rows(&h->m_o, h->o, d, rows_p, 128);
     ok = ok && map_rows(&h->m_f, h->f, F, rows_p, 128);
+    ok = ok && make_qkv_map(&h->m_qkv, h->qkv, (int)rows_p, d);
     ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
     ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
     if (ph) {
@@ -346,8 +352,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.epi.bias = h->qkv_b[l]; g.epi.out = h->qkv; g.epi.ldo = 3 * d;
     ENC_RUN(ENC_K_QKV, 6.0 * Rd * d, launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s));
     ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d,
-            launch_attention_bf16(reinterpret_cast<const bf16*>(h->qkv), reinterpret_cast<bf16*>(h->o), cu, B,
-                                  wk.max_n, d, c.n_heads, s));
+            launch_attention_tc(h->m_qkv, reinterpret_cast<bf16*>(h->o), cu, B, wk.max_n, d, c.n_heads, h->status, s));
     g.N = d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->o_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
@@ -713,7 +718,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   float* s_x = h->x;
   int* s_meta = h->meta;
   const CUtensorMap s_conv1_a = h->m_conv1_a, s_conv2_a = h->m_conv2_a, s_ma = h->m_a, s_mo = h->m_o,
-                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1;
+                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mqkv = h->m_qkv;
   const bool s_profile = h->profile;
   h->melT = melT; h->y1 = y1; h->x = reinterpret_cast<float*>(x); h->a = a; h->qkv = qkv; h->o = o; h->f = f;
   h->e = e; h->p1 = p1; h->meta = reinterpret_cast<int*>(meta);
@@ -725,6 +730,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
     ok = ok && map_rows(&h->m_a, a, d, R, 128);
     ok = ok && map_rows(&h->m_o, o, d, R, 128);
     ok = ok && map_rows(&h->m_f, f, F, R, 128);
+    ok = ok && make_qkv_map(&h->m_qkv, qkv, R, d);
     if (c.proj_hidden) {
       ok = ok && map_rows(&h->m_e, e, d, R_out > 0 ? R_out : 1, 128);
       ok = ok && map_rows(&h->m_p1, p1, c.proj_hidden, R_out > 0 ? R_out : 1, 128);
@@ -745,6 +751,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   h->p1 = s_p1; h->meta = s_meta;
   h->m_conv1_a = s_conv1_a; h->m_conv2_a = s_conv2_a; h->m_a = s_ma; h->m_o = s_mo; h->m_f = s_mf; h->m_e = s_me;
   h->m_p1 = s_mp1;
+  h->m_qkv = s_mqkv;
   h->profile = s_profile;
   return st;
 }

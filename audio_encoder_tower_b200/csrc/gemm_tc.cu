@@ -58,6 +58,50 @@ __device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, 
   }
 }
 
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
+// x[r, n0 .. n0+BN) += acc + bias for one accumulator row per thread. The fp32
+// residual is read four 32-column chunks at a time, all loads issued before the
+// matching TMEM reads, so each group pays one memory latency.
+template <int BN>
+__device__ __forceinline__ void epi_residual_tile(const EpiParams& e, bool row_ok, int r, int n0, uint32_t taddr) {
+  constexpr int G = 4;
+  float* xr = e.resid + (size_t)(row_ok ? r : 0) * e.ldo + n0;
+  const float* br = e.bias ? e.bias + n0 : nullptr;
+#pragma unroll
+  for (int g = 0; g < BN / 32; g += G) {
+    float4 rr[G][8];
+    if (row_ok) {
+#pragma unroll
+      for (int j = 0; j < G; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rr[j][i] = __ldcg(reinterpret_cast<const float4*>(xr + (g + j) * 32) + i);
+    }
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((g + j) * 32), v);
+      tmem_wait_ld();
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (br) b = __ldg(reinterpret_cast<const float4*>(br + (g + j) * 32) + i);
+          float4 o = rr[j][i];
+          o.x += __uint_as_float(v[4 * i]) + b.x;
+          o.y += __uint_as_float(v[4 * i + 1]) + b.y;
+          o.z += __uint_as_float(v[4 * i + 2]) + b.z;
+          o.w += __uint_as_float(v[4 * i + 3]) + b.w;
+          __stcg(reinterpret_cast<float4*>(xr + (g + j) * 32) + i, o);
+        }
+      }
+    }
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
@@ -159,10 +203,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;          // TMEM lanes this warp may read: 32*quarter ..
+    const bool resid = p.epi.mode == EPI_RESIDUAL;
     int acc = 0;
     uint32_t acc_phase = 0;
+    if (resid && blockIdx.x < p.num_tiles) {   // first tile's residual rows toward L2
+      const int r0 = (blockIdx.x / p.tiles_n) * BM + quarter * 32 + lane;
+      if (r0 < p.M)
+        l2_prefetch(p.epi.resid + (size_t)r0 * p.epi.ldo + (blockIdx.x % p.tiles_n) * BN, BN * 4);
+    }
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
+      if (resid) {   // next tile's residual rows toward L2 while this one drains
+        const int nt = tile + gridDim.x;
+        const int rn = (nt / p.tiles_n) * BM + quarter * 32 + lane;
+        if (nt < p.num_tiles && rn < p.M)
+          l2_prefetch(p.epi.resid + (size_t)rn * p.epi.ldo + (nt % p.tiles_n) * BN, BN * 4);
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
         set_status(p.status, kDevTimeout);
         *abort_v = 1;
@@ -170,16 +226,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       }
       tc_fence_after();
       const int r = m0 + quarter * 32 + lane;
-      int dst = 0, pe_row = 0;
-      bool zero = false;
-      const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if (resid) {
+        epi_residual_tile<BN>(p.epi, r < p.M, r, n0, taddr);
+      } else {
+        int dst = 0, pe_row = 0;
+        bool zero = false;
+        const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
-        tmem_wait_ld();
-        if (row_ok) epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+          tmem_wait_ld();
+          if (row_ok)
+            epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

@@ -44,12 +44,15 @@ enc_status enc_linear_bf16(const void* A, const void* W, const float* bias, void
   return launch_gemm_tc(ma, mb, p, sms, stream) == cudaSuccess ? ENC_OK : ENC_ERR_CUDA;
 }
 
-enc_status enc_attention_bf16(const void* qkv, void* out, const int32_t* cu, int32_t B, int32_t max_n,
-                              int32_t n_heads, cudaStream_t stream) {
-  if (!qkv || !out || !cu || B < 1 || max_n < 0 || n_heads < 1) return ENC_ERR_INVALID_ARG;
+enc_status enc_attention_bf16(const void* qkv, void* out, const int32_t* cu, int32_t rows, int32_t B,
+                              int32_t max_n, int32_t n_heads, int* status, cudaStream_t stream) {
+  if (!qkv || !out || !cu || rows < 1 || B < 1 || B > 65535 || max_n < 0 || n_heads < 1 || n_heads > 65535)
+    return ENC_ERR_INVALID_ARG;
   if (!aligned16(qkv) || !aligned16(out)) return ENC_ERR_INVALID_ARG;
-  return launch_attention_bf16(reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(out), cu, B, max_n,
-                               64 * n_heads, n_heads, stream) == cudaSuccess
+  CUtensorMap map;
+  if (!make_qkv_map(&map, qkv, rows, 64 * n_heads)) return ENC_ERR_CUDA;
+  return launch_attention_tc(map, reinterpret_cast<bf16*>(out), cu, B, max_n, 64 * n_heads, n_heads, status,
+                             stream) == cudaSuccess
              ? ENC_OK
              : ENC_ERR_CUDA;
 }

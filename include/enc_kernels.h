@@ -31,14 +31,20 @@ ENC_API enc_status enc_linear_bf16(const void *A, const void *W, const float *bi
 
 /*
  * Bidirectional multi-head attention, head_dim 64 (Voxtral-Mini-3B-2507
- * "(1) AUDIO ENCODER": 20 heads x 64, MHA), over clips packed row after row:
- *   qkv  bf16 [R, 3d]: q | k | v, head h at columns h*64 of each third
- *   cu   device int32 [B+1]: clip b owns rows cu[b] .. cu[b+1]-1 (its keys)
- *   out  bf16 [R, d] = concat_h softmax(q_h k_h^T / 8) v_h
- * max_n = max_b (cu[b+1] - cu[b]) (host value). d = 64 * n_heads.
+ * "(1) AUDIO ENCODER": 20 heads x 64, MHA), over clips packed row after row,
+ * on the tcgen05 tensor cores:
+ *   qkv  bf16 [rows, 3d]: q | k | v, head h at columns h*64 of each third;
+ *        every row must hold finite values (rows of neighbouring clips are
+ *        read by a clip's last key tile and masked out)
+ *   cu   device int32 [B+1]: clip b owns rows cu[b] .. cu[b+1]-1 (its keys);
+ *        cu[B] <= rows
+ *   out  bf16 [rows, d] = concat_h softmax(q_h k_h^T / 8) v_h on rows < cu[B]
+ * max_n >= max_b (cu[b+1] - cu[b]) (host value). d = 64 * n_heads.
+ * status: device int (may be NULL) set to ENC_ERR_TIMEOUT if a bounded wait
+ * inside the kernel runs out.
  */
-ENC_API enc_status enc_attention_bf16(const void *qkv, void *out, const int32_t *cu, int32_t B, int32_t max_n,
-                                      int32_t n_heads, cudaStream_t stream);
+ENC_API enc_status enc_attention_bf16(const void *qkv, void *out, const int32_t *cu, int32_t rows, int32_t B,
+                                      int32_t max_n, int32_t n_heads, int *status, cudaStream_t stream);
 
 #ifdef __cplusplus
 }
