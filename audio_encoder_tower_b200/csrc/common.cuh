@@ -26,6 +26,24 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752440f));
 }
 
+// GELU for the tensor-core epilogues: x * Phi(x) with Phi(x) = erfc(-x / sqrt 2) / 2,
+// erfc(z) for z >= 0 from the rational approximation of Abramowitz & Stegun,
+// Handbook of Mathematical Functions, eq. 7.1.26 (Hastings):
+//   erfc(z) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),  t = 1 / (1 + p z),
+// absolute error below 1.5e-7. Taking Phi(-|x|) directly keeps the relative
+// accuracy of the small tail values; the result is then rounded to bf16.
+__device__ __forceinline__ float gelu_fast(float x) {
+  const float z = fabsf(x) * 0.70710678118654752440f;
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.0f)));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f), 0.254829592f);
+  float e;   // exp(-z^2) = 2^(-z^2 log2 e)
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-z * z * 1.4426950408889634f));
+  const float q = 0.5f * poly * e;   // Phi(-|x|)
+  return x * (x >= 0.f ? 1.0f - q : q);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -107,6 +125,8 @@ __device__ __forceinline__ bool epi_row(const EpiParams& e, int r, int& dst, int
 template <typename OutT, int n>
 __device__ __forceinline__ void epi_apply_run(const EpiParams& e, int dst, int pe_row, bool zero, int c0,
                                               const float* v) {
+  // bf16 outputs come from the tensor-core path: the approximate GELU is far below bf16 rounding there
+  constexpr bool kFastGelu = sizeof(OutT) == 2;
   if (e.mode == EPI_RESIDUAL) {
     float* x = e.resid + (size_t)dst * e.ldo + c0;
 #pragma unroll
@@ -128,10 +148,17 @@ __device__ __forceinline__ void epi_apply_run(const EpiParams& e, int dst, int p
       float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
       if (e.bias) { b0 = e.bias[c0 + i]; b1 = e.bias[c0 + i + 1]; b2 = e.bias[c0 + i + 2]; b3 = e.bias[c0 + i + 3]; }
       float4 r;
-      r.x = gelu_erf(v[i] + b0) + p.x;
-      r.y = gelu_erf(v[i + 1] + b1) + p.y;
-      r.z = gelu_erf(v[i + 2] + b2) + p.z;
-      r.w = gelu_erf(v[i + 3] + b3) + p.w;
+      if (kFastGelu) {
+        r.x = gelu_fast(v[i] + b0) + p.x;
+        r.y = gelu_fast(v[i + 1] + b1) + p.y;
+        r.z = gelu_fast(v[i + 2] + b2) + p.z;
+        r.w = gelu_fast(v[i + 3] + b3) + p.w;
+      } else {
+        r.x = gelu_erf(v[i] + b0) + p.x;
+        r.y = gelu_erf(v[i + 1] + b1) + p.y;
+        r.z = gelu_erf(v[i + 2] + b2) + p.z;
+        r.w = gelu_erf(v[i + 3] + b3) + p.w;
+      }
       *reinterpret_cast<float4*>(x + i) = r;
     }
     return;
@@ -142,7 +169,7 @@ __device__ __forceinline__ void epi_apply_run(const EpiParams& e, int dst, int p
 #pragma unroll
   for (int i = 0; i < n; ++i) {
     float a = v[i] + (e.bias ? e.bias[c0 + i] : 0.f);
-    a = g ? gelu_erf(a) : a;
+    a = g ? (kFastGelu ? gelu_fast(a) : gelu_erf(a)) : a;
     t[i] = zero ? 0.f : a;
   }
   OutT* o = reinterpret_cast<OutT*>(e.out) + (size_t)dst * e.ldo + c0;

@@ -10,7 +10,8 @@
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16)
 //               into a double-buffered TMEM accumulator (2 x BN columns) and
 //               frees ring slots / publishes finished tiles with tcgen05.commit.
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (one row per thread),
+//   warps 2..9  epilogue: tcgen05.ld the accumulator (one row per thread;
+//               warps w and w+4 share TMEM lanes and split the columns),
 //               apply bias / GELU / residual / position-table / scatter, store.
 // The epilogue of tile i overlaps the MMAs of tile i+1.
 //
@@ -30,7 +31,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, each with half of the tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
@@ -63,16 +64,16 @@ __device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
                : "memory");
 }
 
-// x[r, n0 .. n0+BN) += acc + bias for one accumulator row per thread. The fp32
-// residual is read four 32-column chunks at a time, all loads issued before the
-// matching TMEM reads, so each group pays one memory latency.
-template <int BN>
+// x[r, n0 .. n0+32*NC) += acc + bias for one accumulator row per thread. The
+// fp32 residual is read two 32-column chunks at a time, all loads issued before
+// the matching TMEM reads, so each group pays one memory latency.
+template <int NC>
 __device__ __forceinline__ void epi_residual_tile(const EpiParams& e, bool row_ok, int r, int n0, uint32_t taddr) {
-  constexpr int G = 4;
+  constexpr int G = 2;
   float* xr = e.resid + (size_t)(row_ok ? r : 0) * e.ldo + n0;
   const float* br = e.bias ? e.bias + n0 : nullptr;
 #pragma unroll
-  for (int g = 0; g < BN / 32; g += G) {
+  for (int g = 0; g < NC; g += G) {
     float4 rr[G][8];
     if (row_ok) {
 #pragma unroll
@@ -202,22 +203,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    constexpr int NC = BN / 64;            // 32-column chunks per epilogue warp
     const int quarter = warp & 3;          // TMEM lanes this warp may read: 32*quarter ..
+    const int half = (warp - 2) >> 2;      // which half of the tile's columns
     const bool resid = p.epi.mode == EPI_RESIDUAL;
     int acc = 0;
     uint32_t acc_phase = 0;
     if (resid && blockIdx.x < p.num_tiles) {   // first tile's residual rows toward L2
       const int r0 = (blockIdx.x / p.tiles_n) * BM + quarter * 32 + lane;
       if (r0 < p.M)
-        l2_prefetch(p.epi.resid + (size_t)r0 * p.epi.ldo + (blockIdx.x % p.tiles_n) * BN, BN * 4);
+        l2_prefetch(p.epi.resid + (size_t)r0 * p.epi.ldo + (blockIdx.x % p.tiles_n) * BN + half * (BN / 2), BN * 2);
     }
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
+      const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN + half * (BN / 2);
       if (resid) {   // next tile's residual rows toward L2 while this one drains
         const int nt = tile + gridDim.x;
         const int rn = (nt / p.tiles_n) * BM + quarter * 32 + lane;
         if (nt < p.num_tiles && rn < p.M)
-          l2_prefetch(p.epi.resid + (size_t)rn * p.epi.ldo + (nt % p.tiles_n) * BN, BN * 4);
+          l2_prefetch(p.epi.resid + (size_t)rn * p.epi.ldo + (nt % p.tiles_n) * BN + half * (BN / 2), BN * 2);
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
         set_status(p.status, kDevTimeout);
@@ -226,15 +229,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       }
       tc_fence_after();
       const int r = m0 + quarter * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
       if (resid) {
-        epi_residual_tile<BN>(p.epi, r < p.M, r, n0, taddr);
+        epi_residual_tile<NC>(p.epi, r < p.M, r, n0, taddr);
       } else {
         int dst = 0, pe_row = 0;
         bool zero = false;
         const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
           tmem_wait_ld();
