@@ -14,7 +14,9 @@
 //   warp 1      MMA issuer: S_j = Q K_j^T (M=128, N=128, K=64) into one of two
 //               TMEM score buffers, then O += P_j V_j with P_j read from TMEM
 //               (A operand in tensor memory) and V_j from shared memory.
-//   warps 2..5  softmax, one query row per thread (its TMEM lane): row max,
+//   warps 2..9  softmax: two threads per query row (the row's TMEM lane), each
+//               owning 64 of the tile's 128 keys, holding its scores in
+//               registers; the two half-row maxima meet in shared memory.
 //               exp2, row sum, P_j = bf16 into TMEM; the output accumulator O
 //               is rescaled only when a row's running maximum grows by more
 //               than 2^8 (otherwise the stale maximum is kept: P <= 256).
@@ -30,14 +32,15 @@ namespace enc {
 namespace {
 
 constexpr int kQT = 128, kKT = 128, kHD = 64, kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftWarps;
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 320;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
-constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + 2 * kStages) + 256;
+constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + 2 * kStages) + 256 + 2 * 2 * 128 * 4 + 2 * 128 * 4;
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -116,8 +119,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
   uint64_t* p_full = s_empty + 2;                 // [2]
   uint64_t* pv_done = p_full + 2;                 // [2]
   uint64_t* drain = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* red_bar = drain + 1;                  // [2] half-row maxima written
+  uint64_t* sum_bar = red_bar + 2;                // half-row sums written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sum_bar + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* red_max = reinterpret_cast<float*>(bars + 32);   // [2 tiles][2 halves][128 rows]
+  float* red_sum = red_max + 2 * 2 * 128;                  // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -125,11 +132,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     for (int s = 0; s < kStages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_empty[i], 32 * kSoftWarps);
+      mbar_init(&p_full[i], 32 * kSoftWarps);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(&red_bar[0], 32 * kSoftWarps);
+    mbar_init(&red_bar[1], 32 * kSoftWarps);
+    mbar_init(sum_bar, 32 * kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -221,6 +231,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
   } else {
     // ----------------------------------------------------------- softmax
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;      // keys [64*half, 64*half + 64) of each tile
     const int row = quarter * 32 + lane;   // query row inside the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
@@ -229,19 +240,28 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
       const int sb = j & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_v, kWaitNs))) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(sb * kKT);
-      const int kvalid = n - j * kKT;   // keys of this tile that belong to the clip
+      const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(sb * kKT + 64 * half);
+      uint32_t v[64];
+      tmem_ld_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld_32x32b_x32(tS + 32u, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      const int kvalid = n - j * kKT - 64 * half;   // keys of this half-tile inside the clip
+      const bool full = kvalid >= 64;
       float mx = -INFINITY;
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tS + static_cast<uint32_t>(32 * c), v);
-        tmem_wait_ld();
+        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+      } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (32 * c + e < kvalid) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int e = 0; e < 64; ++e)
+          if (e < kvalid) mx = fmaxf(mx, __uint_as_float(v[e]));
       }
-      mx *= scale_log2;
+      // the other half of the row (slot sb is rewritten two tiles later, after
+      // both threads of the row have passed the next tile's exchange)
+      red_max[(sb * 2 + half) * 128 + row] = mx;
+      mbar_arrive(&red_bar[sb]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&red_bar[sb], (j >> 1) & 1u, abort_v, kWaitNs))) { ok = false; break; }
+      mx = fmaxf(mx, red_max[(sb * 2 + (half ^ 1)) * 128 + row]) * scale_log2;
       if (j == 0) {
         m_run = mx;
       } else {
@@ -255,38 +275,40 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
           tc_fence_after();
           const float alpha = need ? ex2(m_run - mx) : 1.f;
           if (need) { m_run = mx; l_run *= alpha; }
+          uint32_t o[32];
+          const uint32_t tO = tmem + lane_off + kColO + static_cast<uint32_t>(32 * half);
+          tmem_ld_32x32b_x32(tO, o);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kHD / 32; ++c) {
-            uint32_t o[32];
-            const uint32_t tO = tmem + lane_off + kColO + static_cast<uint32_t>(32 * c);
-            tmem_ld_32x32b_x32(tO, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st_32x32b_x32(tO, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st_32x32b_x32(tO, o);
           tmem_wait_st();
         }
       }
       // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs into TMEM
-      const uint32_t tP = tmem + lane_off + kColP + static_cast<uint32_t>(sb * (kKT / 2));
+      const uint32_t tP = tmem + lane_off + kColP + static_cast<uint32_t>(sb * (kKT / 2) + 32 * half);
       const float neg_m = -m_run;
+      uint32_t pk[32];
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        uint32_t v[32], pk[16];
-        tmem_ld_32x32b_x32(tS + static_cast<uint32_t>(32 * c), v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, neg_m));
-          float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, neg_m));
-          if (32 * c + e >= kvalid) p0 = 0.f;
-          if (32 * c + e + 1 >= kvalid) p1 = 0.f;
+        for (int e = 0; e < 64; e += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, neg_m));
           l_run += p0 + p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st_32x32b_x16(tP + static_cast<uint32_t>(16 * c), pk);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, neg_m));
+          float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, neg_m));
+          if (e >= kvalid) p0 = 0.f;
+          if (e + 1 >= kvalid) p1 = 0.f;
+          l_run += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
       }
+      tmem_st_32x32b_x32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&s_empty[sb]);
@@ -294,29 +316,30 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1u, abort_v, kWaitNs)))
       ok = false;
-    if (!ok) {
+    // the row sum is split between the two halves
+    red_sum[half * 128 + row] = l_run;
+    mbar_arrive(sum_bar);
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(sum_bar, 0, abort_v, kWaitNs))) ok = false;
+    if (!__all_sync(0xffffffffu, ok)) {
       set_status(status, kDevTimeout);
       *abort_v = 1;
     } else {
       tc_fence_after();
-      const float inv = 1.f / l_run;
+      const float inv = 1.f / (l_run + red_sum[(half ^ 1) * 128 + row]);
       const bool valid = q0 + row < n;
-      bf16* orow = out + (size_t)(start + q0 + row) * d + h * kHD;
+      bf16* orow = out + (size_t)(start + q0 + row) * d + h * kHD + 32 * half;
+      uint32_t o[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + kColO + static_cast<uint32_t>(32 * half), o);
+      tmem_wait_ld();
+      if (valid) {
 #pragma unroll
-      for (int c = 0; c < kHD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_32x32b_x32(tmem + lane_off + kColO + static_cast<uint32_t>(32 * c), o);
-        tmem_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c + e) = u;
-          }
+        for (int e = 0; e < 32; e += 8) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+          u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+          u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + e) = u;
         }
       }
     }
