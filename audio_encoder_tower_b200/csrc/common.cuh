@@ -163,30 +163,32 @@ __device__ __forceinline__ void epi_apply_run(const EpiParams& e, int dst, int p
     }
     return;
   }
-  // EPI_STORE, EPI_CONV1, EPI_SCATTER: value -> OutT
+  // EPI_STORE, EPI_CONV1, EPI_SCATTER: value -> OutT, G columns at a time
+  constexpr int G = n < 8 ? n : 8;   // bf16 stores need 8 columns (16 bytes); fp32 stores take 4
+  static_assert(n % G == 0 && (sizeof(OutT) == 4 || G == 8), "epilogue run width");
   const bool g = e.gelu || e.mode == EPI_CONV1;
-  float t[n];
-#pragma unroll
-  for (int i = 0; i < n; ++i) {
-    float a = v[i] + (e.bias ? e.bias[c0 + i] : 0.f);
-    a = g ? (kFastGelu ? gelu_fast(a) : gelu_erf(a)) : a;
-    t[i] = zero ? 0.f : a;
-  }
   OutT* o = reinterpret_cast<OutT*>(e.out) + (size_t)dst * e.ldo + c0;
-  if constexpr (sizeof(OutT) == 2) {
 #pragma unroll
-    for (int i = 0; i < n; i += 8) {
-      uint4 u;
-      u.x = pack_bf16x2(t[i], t[i + 1]);
-      u.y = pack_bf16x2(t[i + 2], t[i + 3]);
-      u.z = pack_bf16x2(t[i + 4], t[i + 5]);
-      u.w = pack_bf16x2(t[i + 6], t[i + 7]);
-      *reinterpret_cast<uint4*>(o + i) = u;
+  for (int i0 = 0; i0 < n; i0 += G) {
+    float t[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      float a = v[i0 + i] + (e.bias ? e.bias[c0 + i0 + i] : 0.f);
+      a = g ? (kFastGelu ? gelu_fast(a) : gelu_erf(a)) : a;
+      t[i] = zero ? 0.f : a;
     }
-  } else {
+    if constexpr (sizeof(OutT) == 2) {
+      uint4 u;
+      u.x = pack_bf16x2(t[0], t[1]);
+      u.y = pack_bf16x2(t[2], t[3]);
+      u.z = pack_bf16x2(t[4], t[5]);
+      u.w = pack_bf16x2(t[6], t[7]);
+      *reinterpret_cast<uint4*>(o + i0) = u;
+    } else {
 #pragma unroll
-    for (int i = 0; i < n; i += 4)
-      *reinterpret_cast<float4*>(o + i) = make_float4(t[i], t[i + 1], t[i + 2], t[i + 3]);
+      for (int i = 0; i < G; i += 4)
+        *reinterpret_cast<float4*>(o + i0 + i) = make_float4(t[i], t[i + 1], t[i + 2], t[i + 3]);
+    }
   }
 }
 

@@ -54,7 +54,7 @@ struct enc_handle {
   cudaEvent_t meta_free = nullptr;
   bool meta_pending = false;
   // tensor maps (bf16 path)
-  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_qkv;
+  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_qkv, m_x;
   CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
   std::vector<LayerMaps> lmaps;
   // profiling
@@ -250,6 +250,7 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ok = ok && map_rows(&h->m_o, h->o, d, rows_p, 128);
     ok = ok && map_rows(&h->m_f, h->f, F, rows_p, 128);
     ok = ok && make_qkv_map(&h->m_qkv, h->qkv, (int)rows_p, d);
+    ok = ok && make_resid_map(&h->m_x, h->x, (uint64_t)rows_p, (uint64_t)d);
     ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
     ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
     if (ph) {
@@ -356,7 +357,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.N = d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->o_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
-    ENC_RUN(ENC_K_OUT, 2.0 * Rd * d, launch_gemm_tc(h->m_o, lm.o, g, h->sm_count, s));
+    ENC_RUN(ENC_K_OUT, 2.0 * Rd * d, launch_gemm_tc(h->m_o, lm.o, g, h->sm_count, s, &h->m_x));
     ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<bf16>(h->x, h->ln2_g[l], h->ln2_b[l], a, R, d, c.ln_eps, s));
     g.N = F; g.num_kb = d / 64;
     g.epi = epi_base(EPI_STORE);
@@ -365,7 +366,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.N = d; g.num_kb = F / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->fc2_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
-    ENC_RUN(ENC_K_FC2, 2.0 * Rd * F, launch_gemm_tc(h->m_f, lm.fc2, g, h->sm_count, s));
+    ENC_RUN(ENC_K_FC2, 2.0 * Rd * F, launch_gemm_tc(h->m_f, lm.fc2, g, h->sm_count, s, &h->m_x));
   }
 
   if (!c.proj_hidden) {
@@ -718,7 +719,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   float* s_x = h->x;
   int* s_meta = h->meta;
   const CUtensorMap s_conv1_a = h->m_conv1_a, s_conv2_a = h->m_conv2_a, s_ma = h->m_a, s_mo = h->m_o,
-                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mqkv = h->m_qkv;
+                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mqkv = h->m_qkv, s_mx = h->m_x;
   const bool s_profile = h->profile;
   h->melT = melT; h->y1 = y1; h->x = reinterpret_cast<float*>(x); h->a = a; h->qkv = qkv; h->o = o; h->f = f;
   h->e = e; h->p1 = p1; h->meta = reinterpret_cast<int*>(meta);
@@ -731,6 +732,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
     ok = ok && map_rows(&h->m_o, o, d, R, 128);
     ok = ok && map_rows(&h->m_f, f, F, R, 128);
     ok = ok && make_qkv_map(&h->m_qkv, qkv, R, d);
+    ok = ok && make_resid_map(&h->m_x, reinterpret_cast<float*>(x), (uint64_t)R, (uint64_t)d);
     if (c.proj_hidden) {
       ok = ok && map_rows(&h->m_e, e, d, R_out > 0 ? R_out : 1, 128);
       ok = ok && map_rows(&h->m_p1, p1, c.proj_hidden, R_out > 0 ? R_out : 1, 128);
@@ -752,6 +754,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   h->m_conv1_a = s_conv1_a; h->m_conv2_a = s_conv2_a; h->m_a = s_ma; h->m_o = s_mo; h->m_f = s_mf; h->m_e = s_me;
   h->m_p1 = s_mp1;
   h->m_qkv = s_mqkv;
+  h->m_x = s_mx;
   h->profile = s_profile;
   return st;
 }

@@ -42,7 +42,9 @@ struct TcCfg {
   static constexpr uint32_t kBBytes = BN * BK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kTmemCols = 2 * BN;
-  static constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * (size_t)kStageBytes + 256 /*barriers*/;
+  static constexpr size_t kStagingBytes = kEpiWarps * 32 * 32 * 4;   // one 32x32 fp32 tile per epilogue warp
+  static constexpr size_t kSmemBytes =
+      1024 /*align slack*/ + kStages * (size_t)kStageBytes + 1024 /*barriers*/ + kStagingBytes;
 };
 
 __device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, int& x, int& y) {
@@ -59,54 +61,63 @@ __device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, 
   }
 }
 
-__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// x[r, n0 .. n0+32*NC) += acc + bias for one accumulator row per thread. The
-// fp32 residual is read two 32-column chunks at a time, all loads issued before
-// the matching TMEM reads, so each group pays one memory latency.
+// resid[y .. y+32, x .. x+32) += the 32x32 fp32 tile at smem (tensor-map layout,
+// 128-byte swizzle), reduced in L2 by the TMA unit; rows past the map's end are
+// skipped. Completion is tracked with bulk groups.
+__device__ __forceinline__ void tma_reduce_add_2d(const void* map, const void* smem, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// x[r0 .. r0+32, n0 .. n0+32*NC) += acc + bias for the warp's 32 accumulator rows.
+// Each 32-column chunk goes through the warp's 4 KB staging tile: thread = row
+// writes its 32 values (16-byte pieces XOR-swizzled by row, as the tensor map's
+// 128-byte swizzle expects: conflict-free), then one lane hands the tile to the
+// TMA unit as a reduce-add into the fp32 residual, which happens in L2. The SM
+// never loads the residual and nothing here waits on global memory, except for
+// the previous chunk's bulk read of the staging tile.
 template <int NC>
-__device__ __forceinline__ void epi_residual_tile(const EpiParams& e, bool row_ok, int r, int n0, uint32_t taddr) {
-  constexpr int G = 2;
-  float* xr = e.resid + (size_t)(row_ok ? r : 0) * e.ldo + n0;
-  const float* br = e.bias ? e.bias + n0 : nullptr;
+__device__ __forceinline__ void epi_residual_tile(const EpiParams& e, const CUtensorMap* map_c, int r0, int n0,
+                                                  uint32_t taddr, float* tile, int lane) {
+#pragma unroll 1
+  for (int c = 0; c < NC; ++c) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+    if (lane == 0) bulk_wait_read0();   // the previous reduce has read the staging tile
+    tmem_wait_ld();
+    __syncwarp();
+    const float* bias = e.bias ? e.bias + n0 + c * 32 : nullptr;
+    float4* row = reinterpret_cast<float4*>(tile + lane * 32);
 #pragma unroll
-  for (int g = 0; g < NC; g += G) {
-    float4 rr[G][8];
-    if (row_ok) {
-#pragma unroll
-      for (int j = 0; j < G; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) rr[j][i] = __ldcg(reinterpret_cast<const float4*>(xr + (g + j) * 32) + i);
+    for (int j = 0; j < 8; ++j) {
+      const float4 b = bias ? *reinterpret_cast<const float4*>(bias + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      row[j ^ (lane & 7)] = make_float4(__uint_as_float(v[4 * j]) + b.x, __uint_as_float(v[4 * j + 1]) + b.y,
+                                        __uint_as_float(v[4 * j + 2]) + b.z, __uint_as_float(v[4 * j + 3]) + b.w);
     }
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((g + j) * 32), v);
-      tmem_wait_ld();
-      if (row_ok) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (br) b = __ldg(reinterpret_cast<const float4*>(br + (g + j) * 32) + i);
-          float4 o = rr[j][i];
-          o.x += __uint_as_float(v[4 * i]) + b.x;
-          o.y += __uint_as_float(v[4 * i + 1]) + b.y;
-          o.z += __uint_as_float(v[4 * i + 2]) + b.z;
-          o.w += __uint_as_float(v[4 * i + 3]) + b.w;
-          __stcg(reinterpret_cast<float4*>(xr + (g + j) * 32) + i, o);
-        }
-      }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(map_c, tile, n0 + c * 32, r0);
+      bulk_commit();
     }
   }
 }
 
-template <int BN>
+// kResid: the fp32 residual epilogue (EPI_RESIDUAL) is compiled into its own
+// instantiation so that each epilogue keeps the whole register budget.
+template <int BN, bool kResid>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-               const GemmTcParams p) {
+               const __grid_constant__ CUtensorMap map_c, const GemmTcParams p) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -119,6 +130,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   uint64_t* drain = tempty + 2;            // all MMAs of this CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* stage_c = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 1024);   // [kEpiWarps][32 x 32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -206,22 +218,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     constexpr int NC = BN / 64;            // 32-column chunks per epilogue warp
     const int quarter = warp & 3;          // TMEM lanes this warp may read: 32*quarter ..
     const int half = (warp - 2) >> 2;      // which half of the tile's columns
-    const bool resid = p.epi.mode == EPI_RESIDUAL;
     int acc = 0;
     uint32_t acc_phase = 0;
-    if (resid && blockIdx.x < p.num_tiles) {   // first tile's residual rows toward L2
-      const int r0 = (blockIdx.x / p.tiles_n) * BM + quarter * 32 + lane;
-      if (r0 < p.M)
-        l2_prefetch(p.epi.resid + (size_t)r0 * p.epi.ldo + (blockIdx.x % p.tiles_n) * BN + half * (BN / 2), BN * 2);
-    }
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN + half * (BN / 2);
-      if (resid) {   // next tile's residual rows toward L2 while this one drains
-        const int nt = tile + gridDim.x;
-        const int rn = (nt / p.tiles_n) * BM + quarter * 32 + lane;
-        if (nt < p.num_tiles && rn < p.M)
-          l2_prefetch(p.epi.resid + (size_t)rn * p.epi.ldo + (nt % p.tiles_n) * BN + half * (BN / 2), BN * 2);
-      }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
         set_status(p.status, kDevTimeout);
         *abort_v = 1;
@@ -231,8 +231,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       const int r = m0 + quarter * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
-      if (resid) {
-        epi_residual_tile<NC>(p.epi, r < p.M, r, n0, taddr);
+      if constexpr (kResid) {
+        epi_residual_tile<NC>(p.epi, &map_c, m0 + quarter * 32, n0, taddr, stage_c + (warp - 2) * 32 * 32, lane);
       } else {
         int dst = 0, pe_row = 0;
         bool zero = false;
@@ -250,6 +250,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+    }
+    if constexpr (kResid) {
+      if (lane == 0) bulk_wait0();   // the residual reduces have landed
     }
   }
 
@@ -273,19 +276,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int BN>
+template <int BN, bool kResid>
 bool configure_once() {
   static unsigned long long done = 0;   // bit per device ordinal
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(done & bit)) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, kResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)TcCfg<BN>::kSmemBytes) != cudaSuccess)
       return false;
     done |= bit;
   }
   return true;
+}
+
+template <int BN, bool kResid>
+cudaError_t launch_one(const CUtensorMap& map_a, const CUtensorMap& map_b, const CUtensorMap& map_c,
+                       const GemmTcParams& p, int grid, cudaStream_t stream) {
+  if (!configure_once<BN, kResid>()) return cudaErrorInvalidValue;
+  gemm_tc_kernel<BN, kResid><<<grid, kThreads, TcCfg<BN>::kSmemBytes, stream>>>(map_a, map_b, map_c, p);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -307,21 +318,33 @@ bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ro
   return r == CUDA_SUCCESS;
 }
 
+bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (!fn || !resid || (reinterpret_cast<uintptr_t>(resid) & 15u) || ((cols * 4) & 15u)) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(resid), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, const CUtensorMap* map_c) {
   if (p.M <= 0) return cudaSuccess;
   const int bn = gemm_tile_n(p.N);
   p.tiles_n = p.N / bn;
   p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
   const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
-  if (bn == 256) {
-    if (!configure_once<256>()) return cudaErrorInvalidValue;
-    gemm_tc_kernel<256><<<grid, kThreads, TcCfg<256>::kSmemBytes, stream>>>(map_a, map_b, p);
-  } else {
-    if (!configure_once<128>()) return cudaErrorInvalidValue;
-    gemm_tc_kernel<128><<<grid, kThreads, TcCfg<128>::kSmemBytes, stream>>>(map_a, map_b, p);
-  }
-  return cudaGetLastError();
+  const bool resid = p.epi.mode == EPI_RESIDUAL;
+  if (resid && !map_c) return cudaErrorInvalidValue;
+  const CUtensorMap& mc = resid ? *map_c : map_a;
+  if (bn == 256)
+    return resid ? launch_one<256, true>(map_a, map_b, mc, p, grid, stream)
+                 : launch_one<256, false>(map_a, map_b, mc, p, grid, stream);
+  return resid ? launch_one<128, true>(map_a, map_b, mc, p, grid, stream)
+               : launch_one<128, false>(map_a, map_b, mc, p, grid, stream);
 }
 
 }  // namespace enc

@@ -29,8 +29,13 @@ int gemm_tile_n(int n);   // 256 when N % 256 == 0, else 128
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
                  uint32_t box_inner, uint32_t box_rows);
 
+// fp32 [rows, cols] residual matrix as the target of TMA reduce-adds (32 x 32 boxes,
+// 128-byte swizzle). Rows past `rows` are never written.
+bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_t cols);
+
+// map_c: the residual map (EPI_RESIDUAL only; ignored otherwise).
 cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
-                           cudaStream_t stream);
+                           cudaStream_t stream, const CUtensorMap* map_c = nullptr);
 
 // --------------------------------------------------------- fp32 check path
 // C = A[M, K] (row stride lda, rows may overlap) * W[N, K]^T (row stride ldw).
