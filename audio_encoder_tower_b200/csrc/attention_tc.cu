@@ -8,22 +8,26 @@
 // Whisper encoder (Qwen2-Audio-7B-Instruct, "(1) AUDIO ENCODER"; head_dim 64,
 // MHA: Voxtral-Mini-3B-2507, "(1) AUDIO ENCODER").
 //
-// One CTA = 128 query rows of one (clip, head). Warp roles:
-//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
-//               3-stage ring (128-byte swizzle).
-//   warp 1      MMA issuer: S_j = Q K_j^T (M=128, N=128, K=64) into one of two
-//               TMEM score buffers, then O += P_j V_j with P_j read from TMEM
-//               (A operand in tensor memory) and V_j from shared memory.
-//   warps 2..9  softmax: two threads per query row (the row's TMEM lane), each
-//               owning 64 of the tile's 128 keys, holding its scores in
-//               registers; the two half-row maxima meet in shared memory.
-//               exp2, row sum, P_j = bf16 into TMEM; the output accumulator O
-//               is rescaled only when a row's running maximum grows by more
-//               than 2^8 (otherwise the stale maximum is kept: P <= 256).
-//               At the end O / l is written out as bf16.
-// S_{j+1} is computed while the softmax works on S_j.
+// One CTA = two tiles of 128 query rows (A and B) of one (clip, head); both
+// consume the same stream of K/V tiles of 128 keys. Warp roles:
+//   warp 0      TMA: Q_A, Q_B once, then K_j and V_j into a 3-stage ring
+//               (128-byte swizzle).
+//   warp 1      MMA issuer: S_X(j) = Q_X K_j^T (M=128, N=128, K=64) into the
+//               tile's TMEM score buffer, and O_X += P_X(j) V_j with P read from
+//               TMEM (A operand in tensor memory), V_j from shared memory.
+//               Per tile X the order is PV_X(j) then S_X(j+1), so the commit that
+//               publishes S_X(j+1) also guarantees that P_X(j) has been consumed
+//               and O_X holds P_X(j) V_j.
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: one query row
+//               per thread (its TMEM lane), the whole 128-key score row in
+//               registers: row max, exp2, row sum, P = bf16 into TMEM. O is
+//               rescaled only when a row's running maximum grows by more than
+//               2^8 (otherwise the stale maximum is kept: P <= 256). The two
+//               groups run independently, so one group's exponentials overlap
+//               the other's loads and maxima. At the end O / l is stored.
 //
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,320) P0 [320,384) P1 [384,448).
+// TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
+//                     P_A [384,448) P_B [448,512).
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,15 +36,14 @@ namespace enc {
 namespace {
 
 constexpr int kQT = 128, kKT = 128, kHD = 64, kStages = 3;
-constexpr int kSoftWarps = 8;
-constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr int kThreads = 64 + 2 * 128;
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 320;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
-constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + 2 * kStages) + 256 + 2 * 2 * 128 * 4 + 2 * 128 * 4;
+constexpr size_t kSmemBytes = 1024 + kTileBytes * (2 + 2 * kStages) + 256;
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -101,30 +104,25 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
                     int d, float scale_log2, int* status) {
   const int b = blockIdx.z, h = blockIdx.y;
   const int start = cu[b], n = cu[b + 1] - start;
-  const int q0 = blockIdx.x * kQT;
+  const int q0 = blockIdx.x * 2 * kQT;
   if (q0 >= n) return;
   const int nkv = (n + kKT - 1) / kKT;
+  const bool has_b = q0 + kQT < n;   // the second query tile holds rows of the clip
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTileBytes;                  // kStages tiles
+  uint8_t* sQ = smem;                             // 2 tiles: A, B
+  uint8_t* sK = sQ + 2 * kTileBytes;              // kStages tiles
   uint8_t* sV = sK + kStages * kTileBytes;        // kStages tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * kTileBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;          // [2]
-  uint64_t* s_empty = s_full + 2;                 // [2]
-  uint64_t* p_full = s_empty + 2;                 // [2]
-  uint64_t* pv_done = p_full + 2;                 // [2]
-  uint64_t* drain = pv_done + 2;
-  uint64_t* red_bar = drain + 1;                  // [2] half-row maxima written
-  uint64_t* sum_bar = red_bar + 2;                // half-row sums written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sum_bar + 1);
+  uint64_t* s_full = kv_empty + kStages;          // [2] per query tile
+  uint64_t* p_full = s_full + 2;                  // [2] per query tile: S read, P written
+  uint64_t* o_done = p_full + 2;                  // all MMAs of the CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* red_max = reinterpret_cast<float*>(bars + 32);   // [2 tiles][2 halves][128 rows]
-  float* red_sum = red_max + 2 * 2 * 128;                  // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -132,14 +130,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     for (int s = 0; s < kStages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 32 * kSoftWarps);
-      mbar_init(&p_full[i], 32 * kSoftWarps);
-      mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], 128);
     }
-    mbar_init(drain, 1);
-    mbar_init(&red_bar[0], 32 * kSoftWarps);
-    mbar_init(&red_bar[1], 32 * kSoftWarps);
-    mbar_init(sum_bar, 32 * kSoftWarps);
+    mbar_init(o_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -156,8 +149,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     if (lane == 0) {
       bool ok = true;
       uint32_t armed = 0, armed_ph = 0;
-      mbar_arrive_expect_tx(q_full, kTileBytes);
+      mbar_arrive_expect_tx(q_full, (has_b ? 2 : 1) * kTileBytes);
       tma_load_2d(sQ, &map_qkv, q_full, h * kHD, start + q0);
+      if (has_b) tma_load_2d(sQ + kTileBytes, &map_qkv, q_full, h * kHD, start + q0 + kQT);
       int st = 0;
       uint32_t ph = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -182,164 +176,180 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHD) | (1u << 16);   // B (V) MN-major
+      const int ntiles = has_b ? 2 : 1;
       bool ok = mbar_wait(q_full, 0, abort_v, kWaitNs);
       bool issued = false;
-      const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
-      auto issue_s = [&](int j, int stage) {
+      auto issue_s = [&](int x, int stage) {   // S_x = Q_x K^T
+        const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ + x * kTileBytes));
         const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + stage * kTileBytes));
-        const uint32_t dS = tmem + kColS + static_cast<uint32_t>((j & 1) * kKT);
+        const uint32_t dS = tmem + kColS + static_cast<uint32_t>(x * kKT);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k)
           umma_f16_ss(dS, qdesc + static_cast<uint64_t>(2 * k), kdesc + static_cast<uint64_t>(2 * k), idesc_s,
                       k > 0 ? 1u : 0u);
-        umma_commit(&s_full[j & 1]);
+        umma_commit(&s_full[x]);
         issued = true;
+      };
+      auto issue_pv = [&](int x, int stage, int j) {   // O_x += P_x V
+        const uint64_t vdesc = smem_desc_sw128_mn(smem_u32(sV + stage * kTileBytes));
+        const uint32_t aP = tmem + kColP + static_cast<uint32_t>(x * (kKT / 2));
+        const uint32_t dO = tmem + kColO + static_cast<uint32_t>(x * kHD);
+#pragma unroll
+        for (int k = 0; k < kKT / 16; ++k)   // 16 keys per step: 8 TMEM columns of P, 2048 B of V
+          umma_f16_ts(dO, aP + static_cast<uint32_t>(8 * k), vdesc + static_cast<uint64_t>(128 * k), idesc_pv,
+                      (j > 0 || k > 0) ? 1u : 0u);
       };
       int st = 0;
       uint32_t ph = 0;
       if (ok) ok = mbar_wait(&kv_full[0], 0, abort_v, kWaitNs);
-      if (ok) { tc_fence_after(); issue_s(0, 0); }
+      if (ok) {
+        tc_fence_after();
+        for (int x = 0; x < ntiles; ++x) issue_s(x, 0);
+      }
       for (int j = 0; ok && j < nkv; ++j) {
         const int st1 = (st + 1 == kStages) ? 0 : st + 1;
         const uint32_t ph1 = (st + 1 == kStages) ? (ph ^ 1u) : ph;
-        if (j + 1 < nkv) {
-          if (!mbar_wait(&kv_full[st1], ph1, abort_v, kWaitNs)) { ok = false; break; }
-          // the score buffer of tile j+1 was last read by the softmax of tile j-1
-          if (!mbar_wait(&s_empty[(j + 1) & 1], (((j + 1) >> 1) & 1u) ^ 1u, abort_v, kWaitNs)) { ok = false; break; }
+        bool next_ready = false;
+        for (int x = 0; x < ntiles; ++x) {
+          if (!mbar_wait(&p_full[x], j & 1u, abort_v, kWaitNs)) { ok = false; break; }
           tc_fence_after();
-          issue_s(j + 1, st1);
+          issue_pv(x, st, j);
+          if (j + 1 < nkv) {
+            if (!next_ready) {
+              if (!mbar_wait(&kv_full[st1], ph1, abort_v, kWaitNs)) { ok = false; break; }
+              tc_fence_after();
+              next_ready = true;
+            }
+            issue_s(x, st1);   // its commit also covers PV_x(j)
+          }
         }
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1u, abort_v, kWaitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t vdesc = smem_desc_sw128_mn(smem_u32(sV + st * kTileBytes));
-        const uint32_t aP = tmem + kColP + static_cast<uint32_t>((j & 1) * (kKT / 2));
-#pragma unroll
-        for (int k = 0; k < kKT / 16; ++k)   // 16 keys per step: 8 TMEM columns of P, 2048 B of V
-          umma_f16_ts(tmem + kColO, aP + static_cast<uint32_t>(8 * k), vdesc + static_cast<uint64_t>(128 * k),
-                      idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&pv_done[j & 1]);
+        if (!ok) break;
         umma_commit(&kv_empty[st]);
         st = st1;
         ph = ph1;
       }
       if (!ok) { set_status(status, kDevTimeout); *abort_v = 1; }
-      if (issued) {
-        umma_commit(drain);
-        mbar_wait(drain, 0, nullptr, kWaitNs);
+      if (issued) {   // every MMA done: O final, TMEM safe to release
+        umma_commit(o_done);
+        mbar_wait(o_done, 0, nullptr, kWaitNs);
       }
     }
   } else {
     // ----------------------------------------------------------- softmax
+    const int x = (warp - 2) >> 2;          // query tile of this warpgroup
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;      // keys [64*half, 64*half + 64) of each tile
-    const int row = quarter * 32 + lane;   // query row inside the tile = TMEM lane
+    const int row = quarter * 32 + lane;    // query row inside the tile = TMEM lane
+    const int qrow = q0 + x * kQT + row;    // query row inside the clip
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(x * kKT);
+    const uint32_t tO = tmem + lane_off + kColO + static_cast<uint32_t>(x * kHD);
+    const uint32_t tP = tmem + lane_off + kColP + static_cast<uint32_t>(x * (kKT / 2));
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (j >> 1) & 1u, abort_v, kWaitNs))) { ok = false; break; }
+    const bool active = x == 0 || has_b;
+    for (int j = 0; active && j < nkv; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1u, abort_v, kWaitNs))) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(sb * kKT + 64 * half);
-      uint32_t v[64];
-      tmem_ld_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld_32x32b_x32(tS + 32u, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      uint32_t v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld_32x32b_x32(tS + static_cast<uint32_t>(32 * c), *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
       tmem_wait_ld();
-      const int kvalid = n - j * kKT - 64 * half;   // keys of this half-tile inside the clip
-      const bool full = kvalid >= 64;
-      float mx = -INFINITY;
-      if (full) {
+      const int kvalid = n - j * kKT;       // keys of this tile inside the clip
+      const bool full = kvalid >= kKT;
+      float mx;
+      {   // eight independent partial maxima, then a tree
+        float pm[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
-      } else {
+        for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+        if (full) {
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (e < kvalid) mx = fmaxf(mx, __uint_as_float(v[e]));
+          for (int e = 0; e < 128; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e < kvalid) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(v[e]));
+        }
+        mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        mx *= scale_log2;
       }
-      // the other half of the row (slot sb is rewritten two tiles later, after
-      // both threads of the row have passed the next tile's exchange)
-      red_max[(sb * 2 + half) * 128 + row] = mx;
-      mbar_arrive(&red_bar[sb]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&red_bar[sb], (j >> 1) & 1u, abort_v, kWaitNs))) { ok = false; break; }
-      mx = fmaxf(mx, red_max[(sb * 2 + (half ^ 1)) * 128 + row]) * scale_log2;
+      // a row whose maximum grew by more than 2^8 moves to the new maximum; O is
+      // rescaled below, after P is written and before the P.V MMA may start
+      bool rescale = false;
+      float alpha = 1.f;
       if (j == 0) {
         m_run = mx;
       } else {
         const bool need = mx > m_run + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          // O must hold P_{j-1} V_{j-1} before it is rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1u, abort_v, kWaitNs))) {
-            ok = false;
-            break;
+        rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          alpha = ex2(m_run - mx);
+          m_run = mx;
+          l_run *= alpha;
+        }
+      }
+      // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs into TMEM, 32 keys at a time
+      const float neg_m = -m_run;
+      float ps[8];   // eight independent partial row sums
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int k = 32 * c + e;
+          float p0 = ex2(fmaf(__uint_as_float(v[k]), scale_log2, neg_m));
+          float p1 = ex2(fmaf(__uint_as_float(v[k + 1]), scale_log2, neg_m));
+          if (!full) {
+            if (k >= kvalid) p0 = 0.f;
+            if (k + 1 >= kvalid) p1 = 0.f;
           }
-          tc_fence_after();
-          const float alpha = need ? ex2(m_run - mx) : 1.f;
-          if (need) { m_run = mx; l_run *= alpha; }
+          ps[(e >> 1) & 7] += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32b_x16(tP + static_cast<uint32_t>(16 * c), pk);
+      }
+      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (rescale) {   // O_x holds P(j-1) V(j-1): the commit that published S(j) came after that MMA
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
           uint32_t o[32];
-          const uint32_t tO = tmem + lane_off + kColO + static_cast<uint32_t>(32 * half);
-          tmem_ld_32x32b_x32(tO, o);
+          tmem_ld_32x32b_x32(tO + static_cast<uint32_t>(32 * c), o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st_32x32b_x32(tO, o);
-          tmem_wait_st();
+          tmem_st_32x32b_x32(tO + static_cast<uint32_t>(32 * c), o);
         }
       }
-      // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs into TMEM
-      const uint32_t tP = tmem + lane_off + kColP + static_cast<uint32_t>(sb * (kKT / 2) + 32 * half);
-      const float neg_m = -m_run;
-      uint32_t pk[32];
-      if (full) {
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, neg_m));
-          l_run += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, neg_m));
-          float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, neg_m));
-          if (e >= kvalid) p0 = 0.f;
-          if (e + 1 >= kvalid) p1 = 0.f;
-          l_run += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-      }
-      tmem_st_32x32b_x32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&s_empty[sb]);
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[x]);
     }
-    if (ok && !__all_sync(0xffffffffu, mbar_wait(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1u, abort_v, kWaitNs)))
-      ok = false;
-    // the row sum is split between the two halves
-    red_sum[half * 128 + row] = l_run;
-    mbar_arrive(sum_bar);
-    if (ok && !__all_sync(0xffffffffu, mbar_wait(sum_bar, 0, abort_v, kWaitNs))) ok = false;
+    if (active && ok && !__all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_v, kWaitNs))) ok = false;
     if (!__all_sync(0xffffffffu, ok)) {
       set_status(status, kDevTimeout);
       *abort_v = 1;
-    } else {
+    } else if (active) {
       tc_fence_after();
-      const float inv = 1.f / (l_run + red_sum[(half ^ 1) * 128 + row]);
-      const bool valid = q0 + row < n;
-      bf16* orow = out + (size_t)(start + q0 + row) * d + h * kHD + 32 * half;
-      uint32_t o[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + kColO + static_cast<uint32_t>(32 * half), o);
-      tmem_wait_ld();
-      if (valid) {
+      const float inv = 1.f / l_run;
+      const bool valid = qrow < n;
+      bf16* orow = out + (size_t)(start + qrow) * d + h * kHD;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + e) = u;
+      for (int c = 0; c < kHD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + static_cast<uint32_t>(32 * c), o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + e) = u;
+          }
         }
       }
     }
@@ -369,7 +379,7 @@ cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int
     if (e != cudaSuccess) return e;
     done |= 1ull << (dev & 63);
   }
-  dim3 grid((max_n + kQT - 1) / kQT, H, B);
+  dim3 grid((max_n + 2 * kQT - 1) / (2 * kQT), H, B);
   attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map_qkv, out, cu, d, 0.125f * 1.4426950408889634f,
                                                               status);
   return cudaGetLastError();
