@@ -18,13 +18,17 @@
 //               Per tile X the order is PV_X(j) then S_X(j+1), so the commit that
 //               publishes S_X(j+1) also guarantees that P_X(j) has been consumed
 //               and O_X holds P_X(j) V_j.
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: one query row
+//   warps 2, 3  idle (they complete warpgroup 0 for the register split below)
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one query row
 //               per thread (its TMEM lane), the whole 128-key score row in
 //               registers: row max, exp2, row sum, P = bf16 into TMEM. O is
 //               rescaled only when a row's running maximum grows by more than
 //               2^8 (otherwise the stale maximum is kept: P <= 256). The two
 //               groups run independently, so one group's exponentials overlap
 //               the other's loads and maxima. At the end O / l is stored.
+// Registers: launched at 168 per thread (384 threads); warpgroup 0 drops to
+// 88 and the two softmax warpgroups rise to 208 (setmaxnreg), which adds up to
+// exactly the launch total (128*88 + 256*208 = 384*168).
 //
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
 //                     P_A [384,448) P_B [448,512).
@@ -36,7 +40,9 @@ namespace enc {
 namespace {
 
 constexpr int kQT = 128, kKT = 128, kHD = 64, kStages = 3;
-constexpr int kThreads = 64 + 2 * 128;
+constexpr int kThreads = 3 * 128;
+constexpr int kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
+static_assert(128 * kRegsLow + 256 * kRegsHigh == kThreads * kRegsLaunch, "register split must match the launch");
 constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
@@ -143,8 +149,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_v = abort_flag;
-
-  if (warp == 0) {
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+   if (warp == 0) {
     // -------------------------------------------------------------- TMA
     if (lane == 0) {
       bool ok = true;
@@ -171,7 +178,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
           if (armed & (1u << s)) mbar_wait(&kv_full[s], (armed_ph >> s) & 1u, nullptr, kWaitNs / 4);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
@@ -234,9 +241,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
         mbar_wait(o_done, 0, nullptr, kWaitNs);
       }
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     // ----------------------------------------------------------- softmax
-    const int x = (warp - 2) >> 2;          // query tile of this warpgroup
+    const int x = (warp - 4) >> 2;          // query tile of this warpgroup
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;    // query row inside the tile = TMEM lane
     const int qrow = q0 + x * kQT + row;    // query row inside the clip
@@ -374,8 +383,13 @@ cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
   if (!(done & (1ull << (dev & 63)))) {
-    cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    // setmaxnreg redistributes the registers the CTA was launched with: refuse to
+    // launch unless the compiled kernel really holds 168 per thread
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attention_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     done |= 1ull << (dev & 63);
   }
