@@ -8,30 +8,26 @@
 // Whisper encoder (Qwen2-Audio-7B-Instruct, "(1) AUDIO ENCODER"; head_dim 64,
 // MHA: Voxtral-Mini-3B-2507, "(1) AUDIO ENCODER").
 //
-// One CTA = two tiles of 128 query rows (A and B) of one (clip, head); both
-// consume the same stream of K/V tiles of 128 keys. Warp roles:
-//   warp 0      TMA: Q_A, Q_B once, then K_j and V_j into a 3-stage ring
-//               (128-byte swizzle).
-//   warp 1      MMA issuer: S_X(j) = Q_X K_j^T (M=128, N=128, K=64) into the
-//               tile's TMEM score buffer, and O_X += P_X(j) V_j with P read from
-//               TMEM (A operand in tensor memory), V_j from shared memory.
-//               Per tile X the order is PV_X(j) then S_X(j+1), so the commit that
-//               publishes S_X(j+1) also guarantees that P_X(j) has been consumed
-//               and O_X holds P_X(j) V_j.
-//   warps 2, 3  idle (they complete warpgroup 0 for the register split below)
-//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one query row
-//               per thread (its TMEM lane), the whole 128-key score row in
-//               registers: row max, exp2, row sum, P = bf16 into TMEM. O is
+// One CTA = 128 query rows of one (clip, head); two CTAs share an SM, so one
+// CTA's exponentials overlap the other's waits. K/V stream in tiles of 96 keys.
+//   warp 0      TMA: Q once, then K_j and V_j into a 3-stage ring (128-byte swizzle).
+//   warp 1      MMA issuer. S_j = Q K_j^T (M=128, N=96, K=64) goes to score
+//               buffer j%2, so S_{j+1} is ready while the softmax works on S_j.
+//               O += P_j V_j reads P_j from TMEM (A operand in tensor memory):
+//               the softmax writes P_j (bf16) over the first 48 columns of S_j's
+//               own buffer. S_{j+2} reuses that buffer only after P_j V_j has
+//               completed.
+//   warps 2, 3  idle (they complete warpgroup 0 for the register split)
+//   warps 4..7  softmax: one query row per thread (its TMEM lane), the whole
+//               96-key score row in registers: row max, exp2, row sum, P. O is
 //               rescaled only when a row's running maximum grows by more than
-//               2^8 (otherwise the stale maximum is kept: P <= 256). The two
-//               groups run independently, so one group's exponentials overlap
-//               the other's loads and maxima. At the end O / l is stored.
-// Registers: launched at 168 per thread (384 threads); warpgroup 0 drops to
-// 88 and the two softmax warpgroups rise to 208 (setmaxnreg), which adds up to
-// exactly the launch total (128*88 + 256*208 = 384*168).
+//               2^8 (otherwise the stale maximum is kept: P <= 256), after the
+//               previous P V has completed. At the end O / l is stored as bf16.
+// Registers: launched at 128 per thread (256 threads, two CTAs per SM); the
+// control warpgroup drops to 56 and the softmax warpgroup rises to 200
+// (setmaxnreg): 128*56 + 128*200 = 256*128.
 //
-// TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
-//                     P_A [384,448) P_B [448,512).
+// TMEM (256 columns per CTA): S0/P0 [0,96), S1/P1 [96,192), O [192,256).
 #include "common.cuh"
 #include "internal.h"
 
@@ -39,17 +35,18 @@ namespace enc {
 
 namespace {
 
-constexpr int kQT = 128, kKT = 128, kHD = 64, kStages = 3;
-constexpr int kThreads = 3 * 128;
-constexpr int kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
-static_assert(128 * kRegsLow + 256 * kRegsHigh == kThreads * kRegsLaunch, "register split must match the launch");
-constexpr uint32_t kTileBytes = 128 * 64 * 2;   // one 128 x 64 bf16 tile
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr int kQT = 128, kKT = 96, kHD = 64, kStages = 3;
+constexpr int kThreads = 256;
+// registers per thread: launch / control warpgroup / softmax warpgroup (setmaxnreg)
+constexpr int kRegsLaunch = 128, kRegsLow = 56, kRegsHigh = 200;
+static_assert(128 * kRegsLow + 128 * kRegsHigh == kThreads * kRegsLaunch, "register split must match the launch");
+constexpr uint32_t kQBytes = kQT * kHD * 2;      // 16 KB
+constexpr uint32_t kKVBytes = kKT * kHD * 2;     // 12 KB
+constexpr uint32_t kTmemCols = 256;              // two CTAs share an SM's 512 columns
+constexpr uint32_t kColS = 0, kColO = 2 * kKT;   // S buffers [0,96) [96,192), O [192,256)
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr float kRescaleThreshold = 8.0f;       // log2 units
-
-constexpr size_t kSmemBytes = 1024 + kTileBytes * (2 + 2 * kStages) + 256;
+constexpr float kRescaleThreshold = 8.0f;        // log2 units
+constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kKVBytes + 256;
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -105,28 +102,28 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
-attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restrict__ out, const int* __restrict__ cu,
-                    int d, float scale_log2, int* status) {
+__global__ void __launch_bounds__(kThreads, 2)
+attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                    bf16* __restrict__ out, const int* __restrict__ cu, int d, float scale_log2, int* status) {
   const int b = blockIdx.z, h = blockIdx.y;
   const int start = cu[b], n = cu[b + 1] - start;
-  const int q0 = blockIdx.x * 2 * kQT;
+  const int q0 = blockIdx.x * kQT;
   if (q0 >= n) return;
   const int nkv = (n + kKT - 1) / kKT;
-  const bool has_b = q0 + kQT < n;   // the second query tile holds rows of the clip
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                             // 2 tiles: A, B
-  uint8_t* sK = sQ + 2 * kTileBytes;              // kStages tiles
-  uint8_t* sV = sK + kStages * kTileBytes;        // kStages tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * kTileBytes);
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + kQBytes;                     // kStages tiles of 96 keys
+  uint8_t* sV = sK + kStages * kKVBytes;          // kStages tiles of 96 keys
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * kKVBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;          // [2] per query tile
-  uint64_t* p_full = s_full + 2;                  // [2] per query tile: S read, P written
-  uint64_t* o_done = p_full + 2;                  // all MMAs of the CTA complete
+  uint64_t* s_full = kv_empty + kStages;          // [2] score buffer j%2 holds S_j
+  uint64_t* p_full = s_full + 2;                  // [2] softmax read S_j and wrote P_j
+  uint64_t* pv_done = p_full + 2;                 // [2] P_j V_j complete
+  uint64_t* o_done = pv_done + 2;                 // every MMA of the CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -137,103 +134,89 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
     }
     mbar_init(o_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&map_qkv);
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&map_q); tma_prefetch_desc(&map_kv); }
   if (warp == 1) { tmem_alloc(tmem_slot, kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  // K/V tile t sits in ring slot t % kStages, filled for the (t / kStages)-th time
+  auto slot = [](int t) { return t % kStages; };
+  auto fill_parity = [](int t) { return static_cast<uint32_t>((t / kStages) & 1); };
+
   if (warp < 4) {
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-   if (warp == 0) {
-    // -------------------------------------------------------------- TMA
-    if (lane == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA
       bool ok = true;
-      uint32_t armed = 0, armed_ph = 0;
-      mbar_arrive_expect_tx(q_full, (has_b ? 2 : 1) * kTileBytes);
-      tma_load_2d(sQ, &map_qkv, q_full, h * kHD, start + q0);
-      if (has_b) tma_load_2d(sQ + kTileBytes, &map_qkv, q_full, h * kHD, start + q0 + kQT);
-      int st = 0;
-      uint32_t ph = 0;
+      int armed_upto = 0;   // tiles whose loads were issued
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      tma_load_2d(sQ, &map_q, q_full, h * kHD, start + q0);
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_v, kWaitNs)) { ok = false; break; }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * kTileBytes);
-        tma_load_2d(sK + st * kTileBytes, &map_qkv, &kv_full[st], d + h * kHD, start + j * kKT);
-        tma_load_2d(sV + st * kTileBytes, &map_qkv, &kv_full[st], 2 * d + h * kHD, start + j * kKT);
-        armed |= 1u << st;
-        armed_ph = (armed_ph & ~(1u << st)) | (ph << st);
-        if (++st == kStages) { st = 0; ph ^= 1u; }
+        const int st = slot(j);
+        if (!mbar_wait(&kv_empty[st], fill_parity(j) ^ 1u, abort_v, kWaitNs)) { ok = false; break; }
+        mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
+        tma_load_2d(sK + st * kKVBytes, &map_kv, &kv_full[st], d + h * kHD, start + j * kKT);
+        tma_load_2d(sV + st * kKVBytes, &map_kv, &kv_full[st], 2 * d + h * kHD, start + j * kKT);
+        armed_upto = j + 1;
       }
       if (!ok) {
         set_status(status, kDevTimeout);
         *abort_v = 1;
+        // let copies already in flight land before the shared memory goes away
         mbar_wait(q_full, 0, nullptr, kWaitNs / 4);
-        for (int s = 0; s < kStages; ++s)
-          if (armed & (1u << s)) mbar_wait(&kv_full[s], (armed_ph >> s) & 1u, nullptr, kWaitNs / 4);
+        for (int t = armed_upto - kStages; t < armed_upto; ++t)
+          if (t >= 0) mbar_wait(&kv_full[slot(t)], fill_parity(t), nullptr, kWaitNs / 4);
       }
-    }
-   } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHD) | (1u << 16);   // B (V) MN-major
-      const int ntiles = has_b ? 2 : 1;
       bool ok = mbar_wait(q_full, 0, abort_v, kWaitNs);
       bool issued = false;
-      auto issue_s = [&](int x, int stage) {   // S_x = Q_x K^T
-        const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ + x * kTileBytes));
-        const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + stage * kTileBytes));
-        const uint32_t dS = tmem + kColS + static_cast<uint32_t>(x * kKT);
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
+      auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j % 2
+        const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + slot(j) * kKVBytes));
+        const uint32_t dS = tmem + kColS + static_cast<uint32_t>((j & 1) * kKT);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k)
           umma_f16_ss(dS, qdesc + static_cast<uint64_t>(2 * k), kdesc + static_cast<uint64_t>(2 * k), idesc_s,
                       k > 0 ? 1u : 0u);
-        umma_commit(&s_full[x]);
+        umma_commit(&s_full[j & 1]);
         issued = true;
       };
-      auto issue_pv = [&](int x, int stage, int j) {   // O_x += P_x V
-        const uint64_t vdesc = smem_desc_sw128_mn(smem_u32(sV + stage * kTileBytes));
-        const uint32_t aP = tmem + kColP + static_cast<uint32_t>(x * (kKT / 2));
-        const uint32_t dO = tmem + kColO + static_cast<uint32_t>(x * kHD);
-#pragma unroll
-        for (int k = 0; k < kKT / 16; ++k)   // 16 keys per step: 8 TMEM columns of P, 2048 B of V
-          umma_f16_ts(dO, aP + static_cast<uint32_t>(8 * k), vdesc + static_cast<uint64_t>(128 * k), idesc_pv,
-                      (j > 0 || k > 0) ? 1u : 0u);
-      };
-      int st = 0;
-      uint32_t ph = 0;
-      if (ok) ok = mbar_wait(&kv_full[0], 0, abort_v, kWaitNs);
-      if (ok) {
-        tc_fence_after();
-        for (int x = 0; x < ntiles; ++x) issue_s(x, 0);
+      for (int j = 0; ok && j < 2 && j < nkv; ++j) {
+        ok = mbar_wait(&kv_full[slot(j)], fill_parity(j), abort_v, kWaitNs);
+        if (ok) { tc_fence_after(); issue_s(j); }
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        const int st1 = (st + 1 == kStages) ? 0 : st + 1;
-        const uint32_t ph1 = (st + 1 == kStages) ? (ph ^ 1u) : ph;
-        bool next_ready = false;
-        for (int x = 0; x < ntiles; ++x) {
-          if (!mbar_wait(&p_full[x], j & 1u, abort_v, kWaitNs)) { ok = false; break; }
+        const int bf = j & 1;
+        const uint32_t use = static_cast<uint32_t>((j >> 1) & 1);
+        if (!mbar_wait(&p_full[bf], use, abort_v, kWaitNs)) { ok = false; break; }
+        tc_fence_after();
+        // O += P_j V_j: P_j in the first 48 columns of buffer j % 2, 16 keys (8 columns) per step
+        const uint64_t vdesc = smem_desc_sw128_mn(smem_u32(sV + slot(j) * kKVBytes));
+        const uint32_t aP = tmem + kColS + static_cast<uint32_t>(bf * kKT);
+#pragma unroll
+        for (int k = 0; k < kKT / 16; ++k)
+          umma_f16_ts(tmem + kColO, aP + static_cast<uint32_t>(8 * k), vdesc + static_cast<uint64_t>(128 * k),
+                      idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&pv_done[bf]);
+        umma_commit(&kv_empty[slot(j)]);
+        if (j + 2 < nkv) {
+          // S_{j+2} overwrites buffer j % 2: P_j V_j must have read P_j first
+          if (!mbar_wait(&pv_done[bf], use, abort_v, kWaitNs)) { ok = false; break; }
+          if (!mbar_wait(&kv_full[slot(j + 2)], fill_parity(j + 2), abort_v, kWaitNs)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(x, st, j);
-          if (j + 1 < nkv) {
-            if (!next_ready) {
-              if (!mbar_wait(&kv_full[st1], ph1, abort_v, kWaitNs)) { ok = false; break; }
-              tc_fence_after();
-              next_ready = true;
-            }
-            issue_s(x, st1);   // its commit also covers PV_x(j)
-          }
+          issue_s(j + 2);
         }
-        if (!ok) break;
-        umma_commit(&kv_empty[st]);
-        st = st1;
-        ph = ph1;
       }
       if (!ok) { set_status(status, kDevTimeout); *abort_v = 1; }
       if (issued) {   // every MMA done: O final, TMEM safe to release
@@ -241,27 +224,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
         mbar_wait(o_done, 0, nullptr, kWaitNs);
       }
     }
-   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-    // ----------------------------------------------------------- softmax
-    const int x = (warp - 4) >> 2;          // query tile of this warpgroup
+    // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;    // query row inside the tile = TMEM lane
-    const int qrow = q0 + x * kQT + row;    // query row inside the clip
+    const int qrow = q0 + row;              // query row inside the clip
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(x * kKT);
-    const uint32_t tO = tmem + lane_off + kColO + static_cast<uint32_t>(x * kHD);
-    const uint32_t tP = tmem + lane_off + kColP + static_cast<uint32_t>(x * (kKT / 2));
+    const uint32_t tO = tmem + lane_off + kColO;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    const bool active = x == 0 || has_b;
-    for (int j = 0; active && j < nkv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1u, abort_v, kWaitNs))) { ok = false; break; }
+    for (int j = 0; j < nkv; ++j) {
+      const int bf = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[bf], (j >> 1) & 1u, abort_v, kWaitNs))) { ok = false; break; }
       tc_fence_after();
-      uint32_t v[128];
+      const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(bf * kKT);
+      uint32_t v[kKT];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < kKT / 32; ++c)
         tmem_ld_32x32b_x32(tS + static_cast<uint32_t>(32 * c), *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
       tmem_wait_ld();
       const int kvalid = n - j * kKT;       // keys of this tile inside the clip
@@ -273,17 +253,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
         for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
         if (full) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(v[e]));
+          for (int e = 0; e < kKT; ++e) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(v[e]));
         } else {
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
+          for (int e = 0; e < kKT; ++e)
             if (e < kvalid) pm[e & 7] = fmaxf(pm[e & 7], __uint_as_float(v[e]));
         }
         mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         mx *= scale_log2;
       }
-      // a row whose maximum grew by more than 2^8 moves to the new maximum; O is
-      // rescaled below, after P is written and before the P.V MMA may start
+      // a row whose maximum grew by more than 2^8 moves to the new maximum
       bool rescale = false;
       float alpha = 1.f;
       if (j == 0) {
@@ -297,13 +276,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
           l_run *= alpha;
         }
       }
-      // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs into TMEM, 32 keys at a time
+      // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs over the
+      // first 48 columns of this score buffer, 32 keys at a time
       const float neg_m = -m_run;
       float ps[8];   // eight independent partial row sums
 #pragma unroll
       for (int q = 0; q < 8; ++q) ps[q] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kKT / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -317,10 +297,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
           ps[(e >> 1) & 7] += p0 + p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st_32x32b_x16(tP + static_cast<uint32_t>(16 * c), pk);
+        tmem_st_32x32b_x16(tS + static_cast<uint32_t>(16 * c), pk);
       }
       l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      if (rescale) {   // O_x holds P(j-1) V(j-1): the commit that published S(j) came after that MMA
+      if (rescale) {   // O must hold P_{j-1} V_{j-1} before it is scaled
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1u, abort_v, kWaitNs))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < kHD / 32; ++c) {
           uint32_t o[32];
@@ -333,13 +318,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[x]);
+      mbar_arrive(&p_full[bf]);
     }
-    if (active && ok && !__all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_v, kWaitNs))) ok = false;
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(o_done, 0, abort_v, kWaitNs))) ok = false;
     if (!__all_sync(0xffffffffu, ok)) {
       set_status(status, kDevTimeout);
       *abort_v = 1;
-    } else if (active) {
+    } else {
       tc_fence_after();
       const float inv = 1.f / l_run;
       const bool valid = qrow < n;
@@ -372,11 +357,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_qkv, bf16* __restric
   }
 }
 
-bool make_qkv_map(CUtensorMap* map, const void* qkv, int rows, int d) {
-  return make_tma_2d(map, qkv, 3 * (uint64_t)d, (uint64_t)rows, 6 * (uint64_t)d, 64, 128);
+bool make_qkv_maps(QkvMaps* maps, const void* qkv, int rows, int d) {
+  return make_tma_2d(&maps->q, qkv, 3 * (uint64_t)d, (uint64_t)rows, 6 * (uint64_t)d, 64, kQT) &&
+         make_tma_2d(&maps->kv, qkv, 3 * (uint64_t)d, (uint64_t)rows, 6 * (uint64_t)d, 64, kKT);
 }
 
-cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int* cu, int B, int max_n, int d, int H,
+cudaError_t launch_attention_tc(const QkvMaps& maps, bf16* out, const int* cu, int B, int max_n, int d, int H,
                                 int* status, cudaStream_t stream) {
   if (B <= 0 || max_n <= 0) return cudaSuccess;
   static unsigned long long done = 0;
@@ -384,7 +370,7 @@ cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
   if (!(done & (1ull << (dev & 63)))) {
     // setmaxnreg redistributes the registers the CTA was launched with: refuse to
-    // launch unless the compiled kernel really holds 168 per thread
+    // launch unless the compiled kernel holds exactly the planned count per thread
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, attention_tc_kernel);
     if (e != cudaSuccess) return e;
@@ -393,9 +379,9 @@ cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int
     if (e != cudaSuccess) return e;
     done |= 1ull << (dev & 63);
   }
-  dim3 grid((max_n + 2 * kQT - 1) / (2 * kQT), H, B);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map_qkv, out, cu, d, 0.125f * 1.4426950408889634f,
-                                                              status);
+  dim3 grid((max_n + kQT - 1) / kQT, H, B);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.kv, out, cu, d,
+                                                              0.125f * 1.4426950408889634f, status);
   return cudaGetLastError();
 }
 

@@ -54,7 +54,8 @@ struct enc_handle {
   cudaEvent_t meta_free = nullptr;
   bool meta_pending = false;
   // tensor maps (bf16 path)
-  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_qkv, m_x;
+  CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_x;
+  QkvMaps m_qkv;
   CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
   std::vector<LayerMaps> lmaps;
   // profiling
@@ -249,7 +250,7 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ok = ok && map_rows(&h->m_a, h->a, d, rows_p, 128);
     ok = ok && map_rows(&h->m_o, h->o, d, rows_p, 128);
     ok = ok && map_rows(&h->m_f, h->f, F, rows_p, 128);
-    ok = ok && make_qkv_map(&h->m_qkv, h->qkv, (int)rows_p, d);
+    ok = ok && make_qkv_maps(&h->m_qkv, h->qkv, (int)rows_p, d);
     ok = ok && make_resid_map(&h->m_x, h->x, (uint64_t)rows_p, (uint64_t)d);
     ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
     ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
@@ -719,7 +720,8 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   float* s_x = h->x;
   int* s_meta = h->meta;
   const CUtensorMap s_conv1_a = h->m_conv1_a, s_conv2_a = h->m_conv2_a, s_ma = h->m_a, s_mo = h->m_o,
-                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mqkv = h->m_qkv, s_mx = h->m_x;
+                    s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mx = h->m_x;
+  const QkvMaps s_mqkv = h->m_qkv;
   const bool s_profile = h->profile;
   h->melT = melT; h->y1 = y1; h->x = reinterpret_cast<float*>(x); h->a = a; h->qkv = qkv; h->o = o; h->f = f;
   h->e = e; h->p1 = p1; h->meta = reinterpret_cast<int*>(meta);
@@ -731,7 +733,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
     ok = ok && map_rows(&h->m_a, a, d, R, 128);
     ok = ok && map_rows(&h->m_o, o, d, R, 128);
     ok = ok && map_rows(&h->m_f, f, F, R, 128);
-    ok = ok && make_qkv_map(&h->m_qkv, qkv, R, d);
+    ok = ok && make_qkv_maps(&h->m_qkv, qkv, R, d);
     ok = ok && make_resid_map(&h->m_x, reinterpret_cast<float*>(x), (uint64_t)R, (uint64_t)d);
     if (c.proj_hidden) {
       ok = ok && map_rows(&h->m_e, e, d, R_out > 0 ? R_out : 1, 128);

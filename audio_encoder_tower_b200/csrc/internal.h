@@ -46,9 +46,12 @@ cudaError_t launch_sgemm(const float* A, int lda, const float* W, int ldw, int M
 // qkv [R, 3d] packed rows (clip b at rows cu[b] .. cu[b+1]); out [R, d].
 cudaError_t launch_attention_bf16(const bf16* qkv, bf16* out, const int* cu, int B, int max_n, int d, int H,
                                   cudaStream_t stream);
-// tcgen05 attention: map_qkv from make_qkv_map over the same [rows, 3d] buffer.
-bool make_qkv_map(CUtensorMap* map, const void* qkv, int rows, int d);
-cudaError_t launch_attention_tc(const CUtensorMap& map_qkv, bf16* out, const int* cu, int B, int max_n, int d, int H,
+// tcgen05 attention: Q (128-row boxes) and K/V (96-row boxes) views of one [rows, 3d] buffer.
+struct QkvMaps {
+  CUtensorMap q, kv;
+};
+bool make_qkv_maps(QkvMaps* maps, const void* qkv, int rows, int d);
+cudaError_t launch_attention_tc(const QkvMaps& maps, bf16* out, const int* cu, int B, int max_n, int d, int H,
                                 int* status, cudaStream_t stream);
 cudaError_t launch_attention_f32(const float* qkv, float* out, const int* cu, int B, int max_n, int d, int H,
                                  cudaStream_t stream);

@@ -51,9 +51,9 @@ enc_status enc_attention_bf16(const void* qkv, void* out, const int32_t* cu, int
   if (!qkv || !out || !cu || rows < 1 || B < 1 || B > 65535 || max_n < 0 || n_heads < 1 || n_heads > 65535)
     return ENC_ERR_INVALID_ARG;
   if (!aligned16(qkv) || !aligned16(out)) return ENC_ERR_INVALID_ARG;
-  CUtensorMap map;
-  if (!make_qkv_map(&map, qkv, rows, 64 * n_heads)) return ENC_ERR_CUDA;
-  return launch_attention_tc(map, reinterpret_cast<bf16*>(out), cu, B, max_n, 64 * n_heads, n_heads, status,
+  QkvMaps maps;
+  if (!make_qkv_maps(&maps, qkv, rows, 64 * n_heads)) return ENC_ERR_CUDA;
+  return launch_attention_tc(maps, reinterpret_cast<bf16*>(out), cu, B, max_n, 64 * n_heads, n_heads, status,
                              stream) == cudaSuccess
              ? ENC_OK
              : ENC_ERR_CUDA;
