@@ -44,8 +44,6 @@ cudaError_t launch_sgemm(const float* A, int lda, const float* W, int ldw, int M
 
 // ------------------------------------------------------------- attention
 // qkv [R, 3d] packed rows (clip b at rows cu[b] .. cu[b+1]); out [R, d].
-cudaError_t launch_attention_bf16(const bf16* qkv, bf16* out, const int* cu, int B, int max_n, int d, int H,
-                                  cudaStream_t stream);
 // tcgen05 attention: Q (128-row boxes) and K/V (96-row boxes) views of one [rows, 3d] buffer.
 struct QkvMaps {
   CUtensorMap q, kv;
