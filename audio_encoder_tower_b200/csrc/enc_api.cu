@@ -55,6 +55,7 @@ struct enc_handle {
   bool meta_pending = false;
   // tensor maps (bf16 path)
   CUtensorMap m_conv1_a, m_conv2_a, m_a, m_o, m_f, m_e, m_p1, m_x;
+  CUtensorMap m_out_y1, m_out_qkv, m_out_f, m_out_p1;   // bf16 outputs written by TMA stores
   QkvMaps m_qkv;
   CUtensorMap m_conv1_w, m_conv2_w, m_proj1_w, m_proj2_w;
   std::vector<LayerMaps> lmaps;
@@ -252,11 +253,15 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ok = ok && map_rows(&h->m_f, h->f, F, rows_p, 128);
     ok = ok && make_qkv_maps(&h->m_qkv, h->qkv, (int)rows_p, d);
     ok = ok && make_resid_map(&h->m_x, h->x, (uint64_t)rows_p, (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_y1, h->y1, (uint64_t)rows_t, (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_qkv, h->qkv, (uint64_t)rows_p, 3 * (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_f, h->f, (uint64_t)rows_p, (uint64_t)F);
     ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
     ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
     if (ph) {
       ok = ok && map_rows(&h->m_e, h->e, d, rows_o, 128);
       ok = ok && map_rows(&h->m_p1, h->p1, ph, rows_o, 128);
+      ok = ok && make_out_map(&h->m_out_p1, h->p1, (uint64_t)rows_o, (uint64_t)ph);
       ok = ok && map_rows(&h->m_proj1_w, h->proj1_w, d, ph, gemm_tile_n(ph));
       ok = ok && map_rows(&h->m_proj2_w, h->proj2_w, ph, po, gemm_tile_n(po));
     }
@@ -337,7 +342,8 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
   g.M = B * h->Tp; g.N = d; g.a_mode = A_CONV1; g.kb_seg = h->mpad / 64; g.num_kb = 3 * g.kb_seg;
   g.epi = epi_base(EPI_CONV1);
   g.epi.bias = h->conv1_b; g.epi.out = h->y1; g.epi.ldo = d; g.epi.T = h->T; g.epi.Tp = h->Tp;
-  ENC_RUN(ENC_K_CONV1, 2.0 * 2 * Rd * 3 * M, launch_gemm_tc(h->m_conv1_a, h->m_conv1_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_CONV1, 2.0 * 2 * Rd * 3 * M,
+          launch_gemm_tc(h->m_conv1_a, h->m_conv1_w, g, h->sm_count, s, &h->m_out_y1));
   // conv2 (+ GELU + position table) -> packed residual stream
   g.M = B * h->P1; g.N = d; g.a_mode = A_CONV2; g.kb_seg = d / 64; g.num_kb = 3 * g.kb_seg;
   g.epi = epi_base(EPI_CONV2);
@@ -352,7 +358,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.N = 3 * d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_STORE);
     g.epi.bias = h->qkv_b[l]; g.epi.out = h->qkv; g.epi.ldo = 3 * d;
-    ENC_RUN(ENC_K_QKV, 6.0 * Rd * d, launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s));
+    ENC_RUN(ENC_K_QKV, 6.0 * Rd * d, launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s, &h->m_out_qkv));
     ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d,
             launch_attention_tc(h->m_qkv, reinterpret_cast<bf16*>(h->o), cu, B, wk.max_n, d, c.n_heads, h->status, s));
     g.N = d; g.num_kb = d / 64;
@@ -363,7 +369,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.N = F; g.num_kb = d / 64;
     g.epi = epi_base(EPI_STORE);
     g.epi.gelu = 1; g.epi.bias = h->fc1_b[l]; g.epi.out = h->f; g.epi.ldo = F;
-    ENC_RUN(ENC_K_FC1, 2.0 * Rd * F, launch_gemm_tc(h->m_a, lm.fc1, g, h->sm_count, s));
+    ENC_RUN(ENC_K_FC1, 2.0 * Rd * F, launch_gemm_tc(h->m_a, lm.fc1, g, h->sm_count, s, &h->m_out_f));
     g.N = d; g.num_kb = F / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->fc2_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
@@ -385,7 +391,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
   g.N = ph; g.num_kb = d / 64;
   g.epi = epi_base(EPI_STORE);
   g.epi.gelu = 1; g.epi.bias = h->proj1_b; g.epi.out = h->p1; g.epi.ldo = ph;
-  ENC_RUN(ENC_K_PROJ1, 2.0 * Ro * d * ph, launch_gemm_tc(h->m_e, h->m_proj1_w, g, h->sm_count, s));
+  ENC_RUN(ENC_K_PROJ1, 2.0 * Ro * d * ph, launch_gemm_tc(h->m_e, h->m_proj1_w, g, h->sm_count, s, &h->m_out_p1));
   g.N = po; g.num_kb = ph / 64;
   g.epi = epi_base(EPI_SCATTER);
   g.epi.bias = h->proj2_b; g.epi.out = out; g.epi.ldo = po; g.epi.cu = cu_out; g.epi.B = B; g.epi.p_out = h->p_out;
@@ -722,6 +728,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   const CUtensorMap s_conv1_a = h->m_conv1_a, s_conv2_a = h->m_conv2_a, s_ma = h->m_a, s_mo = h->m_o,
                     s_mf = h->m_f, s_me = h->m_e, s_mp1 = h->m_p1, s_mx = h->m_x;
   const QkvMaps s_mqkv = h->m_qkv;
+  const CUtensorMap s_oy1 = h->m_out_y1, s_oqkv = h->m_out_qkv, s_of = h->m_out_f, s_op1 = h->m_out_p1;
   const bool s_profile = h->profile;
   h->melT = melT; h->y1 = y1; h->x = reinterpret_cast<float*>(x); h->a = a; h->qkv = qkv; h->o = o; h->f = f;
   h->e = e; h->p1 = p1; h->meta = reinterpret_cast<int*>(meta);
@@ -735,9 +742,13 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
     ok = ok && map_rows(&h->m_f, f, F, R, 128);
     ok = ok && make_qkv_maps(&h->m_qkv, qkv, R, d);
     ok = ok && make_resid_map(&h->m_x, reinterpret_cast<float*>(x), (uint64_t)R, (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_y1, y1, (uint64_t)rows_t, (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_qkv, qkv, (uint64_t)R, 3 * (uint64_t)d);
+    ok = ok && make_out_map(&h->m_out_f, f, (uint64_t)R, (uint64_t)F);
     if (c.proj_hidden) {
       ok = ok && map_rows(&h->m_e, e, d, R_out > 0 ? R_out : 1, 128);
       ok = ok && map_rows(&h->m_p1, p1, c.proj_hidden, R_out > 0 ? R_out : 1, 128);
+      ok = ok && make_out_map(&h->m_out_p1, p1, (uint64_t)(R_out > 0 ? R_out : 1), (uint64_t)c.proj_hidden);
     }
     if (!ok) st = ENC_ERR_CUDA;
   }
@@ -757,6 +768,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   h->m_p1 = s_mp1;
   h->m_qkv = s_mqkv;
   h->m_x = s_mx;
+  h->m_out_y1 = s_oy1; h->m_out_qkv = s_oqkv; h->m_out_f = s_of; h->m_out_p1 = s_op1;
   h->profile = s_profile;
   return st;
 }

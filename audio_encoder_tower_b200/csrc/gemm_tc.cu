@@ -112,9 +112,68 @@ __device__ __forceinline__ void epi_residual_tile(const EpiParams& e, const CUte
   }
 }
 
-// kResid: the fp32 residual epilogue (EPI_RESIDUAL) is compiled into its own
-// instantiation so that each epilogue keeps the whole register budget.
-template <int BN, bool kResid>
+// out[y .. y+32, x .. x+64) = the 32x64 bf16 tile at smem (tensor-map layout,
+// 128-byte swizzle); rows past the map's end are skipped.
+__device__ __forceinline__ void tma_store_2d(const void* map, const void* smem, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem)), "r"(x), "r"(y)
+               : "memory");
+}
+
+// out[r0 .. r0+32, n0 .. n0+64*NC) = act(acc + bias) as bf16 for the warp's 32
+// accumulator rows (EPI_STORE, EPI_CONV1). Each 64-column chunk is converted
+// into the warp's 4 KB staging tile (thread = row, 16-byte pieces XOR-swizzled
+// by row as the tensor map's 128-byte swizzle expects) and written by one TMA
+// bulk store, so global writes are whole lines and asynchronous.
+template <int NC>
+__device__ __forceinline__ void epi_store_tile(const EpiParams& e, const CUtensorMap* map_c, int r0, int n0,
+                                               uint32_t taddr, uint32_t* tile, int lane) {
+  const int r = r0 + lane;
+  bool zero = false;   // conv1: padding rows of the padded time axis are exact zeros
+  if (e.mode == EPI_CONV1) {
+    const int tp = r % e.Tp;
+    zero = (tp == 0) || (tp > e.T);
+  }
+  const bool g = e.gelu || e.mode == EPI_CONV1;
+#pragma unroll 1
+  for (int c = 0; c < NC; ++c) {
+    uint32_t v[64];
+    tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 64), *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+    tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+    if (lane == 0) bulk_wait_read0();   // the previous store has read the staging tile
+    tmem_wait_ld();
+    __syncwarp();
+    const float* bias = e.bias ? e.bias + n0 + c * 64 : nullptr;
+    uint4* row = reinterpret_cast<uint4*>(tile + lane * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {   // 8 columns -> one 16-byte piece
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float a = __uint_as_float(v[8 * j + i]) + (bias ? bias[8 * j + i] : 0.f);
+        a = g ? gelu_fast(a) : a;
+        t[i] = zero ? 0.f : a;
+      }
+      row[j ^ (lane & 7)] = make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]), pack_bf16x2(t[4], t[5]),
+                                       pack_bf16x2(t[6], t[7]));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map_c, tile, n0 + c * 64, r0);
+      bulk_commit();
+    }
+  }
+}
+
+// Epilogue instantiations: each keeps the whole register budget to itself.
+enum EpiKind : int {
+  EK_GENERIC = 0,   // per-thread stores (conv2 scatter + position table, projector scatter)
+  EK_RESID = 1,     // fp32 residual via TMA reduce-add
+  EK_STORE = 2,     // bf16 output via TMA store (plain rows, conv1)
+};
+template <int BN, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                const __grid_constant__ CUtensorMap map_c, const GemmTcParams p) {
@@ -231,8 +290,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       const int r = m0 + quarter * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
-      if constexpr (kResid) {
+      if constexpr (kEpi == EK_RESID) {
         epi_residual_tile<NC>(p.epi, &map_c, m0 + quarter * 32, n0, taddr, stage_c + (warp - 2) * 32 * 32, lane);
+      } else if constexpr (kEpi == EK_STORE) {
+        epi_store_tile<NC / 2>(p.epi, &map_c, m0 + quarter * 32, n0, taddr,
+                               reinterpret_cast<uint32_t*>(stage_c + (warp - 2) * 32 * 32), lane);
       } else {
         int dst = 0, pe_row = 0;
         bool zero = false;
@@ -251,8 +313,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    if constexpr (kResid) {
-      if (lane == 0) bulk_wait0();   // the residual reduces have landed
+    if constexpr (kEpi != EK_GENERIC) {
+      if (lane == 0) bulk_wait0();   // the bulk stores / reduces have landed
     }
   }
 
@@ -276,14 +338,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int BN, bool kResid>
+template <int BN, int kEpi>
 bool configure_once() {
   static unsigned long long done = 0;   // bit per device ordinal
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(done & bit)) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, kResid>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)TcCfg<BN>::kSmemBytes) != cudaSuccess)
       return false;
     done |= bit;
@@ -291,11 +353,11 @@ bool configure_once() {
   return true;
 }
 
-template <int BN, bool kResid>
+template <int BN, int kEpi>
 cudaError_t launch_one(const CUtensorMap& map_a, const CUtensorMap& map_b, const CUtensorMap& map_c,
                        const GemmTcParams& p, int grid, cudaStream_t stream) {
-  if (!configure_once<BN, kResid>()) return cudaErrorInvalidValue;
-  gemm_tc_kernel<BN, kResid><<<grid, kThreads, TcCfg<BN>::kSmemBytes, stream>>>(map_a, map_b, map_c, p);
+  if (!configure_once<BN, kEpi>()) return cudaErrorInvalidValue;
+  gemm_tc_kernel<BN, kEpi><<<grid, kThreads, TcCfg<BN>::kSmemBytes, stream>>>(map_a, map_b, map_c, p);
   return cudaGetLastError();
 }
 
@@ -316,6 +378,10 @@ bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ro
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_out_map(CUtensorMap* map, const void* out, uint64_t rows, uint64_t cols) {
+  return make_tma_2d(map, out, cols, rows, cols * 2, 64, 32);
 }
 
 bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_t cols) {
@@ -339,12 +405,17 @@ cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, G
   const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
   const bool resid = p.epi.mode == EPI_RESIDUAL;
   if (resid && !map_c) return cudaErrorInvalidValue;
-  const CUtensorMap& mc = resid ? *map_c : map_a;
-  if (bn == 256)
-    return resid ? launch_one<256, true>(map_a, map_b, mc, p, grid, stream)
-                 : launch_one<256, false>(map_a, map_b, mc, p, grid, stream);
-  return resid ? launch_one<128, true>(map_a, map_b, mc, p, grid, stream)
-               : launch_one<128, false>(map_a, map_b, mc, p, grid, stream);
+  // bf16 row outputs go through TMA stores when the caller supplied the output map
+  const bool store = !resid && map_c && (p.epi.mode == EPI_STORE || p.epi.mode == EPI_CONV1);
+  const CUtensorMap& mc = map_c ? *map_c : map_a;
+  if (bn == 256) {
+    if (resid) return launch_one<256, EK_RESID>(map_a, map_b, mc, p, grid, stream);
+    if (store) return launch_one<256, EK_STORE>(map_a, map_b, mc, p, grid, stream);
+    return launch_one<256, EK_GENERIC>(map_a, map_b, mc, p, grid, stream);
+  }
+  if (resid) return launch_one<128, EK_RESID>(map_a, map_b, mc, p, grid, stream);
+  if (store) return launch_one<128, EK_STORE>(map_a, map_b, mc, p, grid, stream);
+  return launch_one<128, EK_GENERIC>(map_a, map_b, mc, p, grid, stream);
 }
 
 }  // namespace enc

@@ -25,6 +25,10 @@ struct GemmTcParams {
 
 int gemm_tile_n(int n);   // 256 when N % 256 == 0, else 128
 
+// bf16 [rows, cols] output matrix as the target of TMA stores (32 x 64 boxes,
+// 128-byte swizzle). Rows past `rows` are never written.
+bool make_out_map(CUtensorMap* map, const void* out, uint64_t rows, uint64_t cols);
+
 // 2-D bf16 tensor map with 128-byte swizzle and zero fill outside the tensor.
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
                  uint32_t box_inner, uint32_t box_rows);
@@ -33,7 +37,8 @@ bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ro
 // 128-byte swizzle). Rows past `rows` are never written.
 bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_t cols);
 
-// map_c: the residual map (EPI_RESIDUAL only; ignored otherwise).
+// map_c: EPI_RESIDUAL: the residual map (required); EPI_STORE / EPI_CONV1: an
+// optional bf16 output map from make_out_map (TMA-store epilogue when given).
 cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
                            cudaStream_t stream, const CUtensorMap* map_c = nullptr);
 

@@ -42,8 +42,9 @@ enc_status enc_linear_bf16(const void* A, const void* W, const float* bias, void
   p.epi.resid = resid;
   p.epi.ldo = N;
   CUtensorMap mc;
-  if (resid && !make_resid_map(&mc, resid, (uint64_t)M, (uint64_t)N)) return ENC_ERR_CUDA;
-  return launch_gemm_tc(ma, mb, p, sms, stream, resid ? &mc : nullptr) == cudaSuccess ? ENC_OK : ENC_ERR_CUDA;
+  if (resid ? !make_resid_map(&mc, resid, (uint64_t)M, (uint64_t)N) : !make_out_map(&mc, out, (uint64_t)M, (uint64_t)N))
+    return ENC_ERR_CUDA;
+  return launch_gemm_tc(ma, mb, p, sms, stream, &mc) == cudaSuccess ? ENC_OK : ENC_ERR_CUDA;
 }
 
 enc_status enc_attention_bf16(const void* qkv, void* out, const int32_t* cu, int32_t rows, int32_t B,
