@@ -46,6 +46,7 @@ constexpr uint32_t kTmemCols = 256;              // two CTAs share an SM's 512 c
 constexpr uint32_t kColS = 0, kColO = 2 * kKT;   // S buffers [0,96) [96,192), O [192,256)
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
+constexpr int kPolyPairs = 1;                    // of every 4 score pairs, this many take exp2_poly2
 constexpr size_t kSmemBytes = 1024 + kQBytes + 2 * kStages * kKVBytes + 256;
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -85,6 +86,46 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (one instruction for two lanes of work on sm_100).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for two values on the FMA pipe (the MUFU unit is the softmax's bottleneck):
+// Cody-Waite split x = n + f, n = round(x) (adding 1.5 * 2^23 rounds to an
+// integer held in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a cubic
+// fitted here for least maximum relative error on [-1/2, 1/2] (7.5e-5, far
+// below the bf16 rounding of P); 2^n enters through the exponent bits. x is
+// clamped at -126 so the exponent never wraps (2^-126 is zero for P).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  constexpr float c0 = 0.99992810936f, c1 = 0.69326098561f, c2 = 0.24261054228f, c3 = 0.05517132143f;
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  add2(t0, t1, x0, x1, kMagic, kMagic);
+  add2(n0, n1, t0, t1, -kMagic, -kMagic);
+  fma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);   // f = x - n
+  fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+  fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  // (bits of t) << 23 == n << 23 modulo 2^32: the 1.5 * 2^23 offset shifts out
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Shared-memory descriptor of a 128-byte-swizzled tile whose rows of 128 B run
@@ -279,7 +320,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs over the
       // first 48 columns of this score buffer, 32 keys at a time
       const float neg_m = -m_run;
-      float ps[8];   // eight independent partial row sums
+      float ps[8];   // eight independent partial row sums (four packed pairs)
 #pragma unroll
       for (int q = 0; q < 8; ++q) ps[q] = 0.f;
 #pragma unroll
@@ -288,13 +329,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int k = 32 * c + e;
-          float p0 = ex2(fmaf(__uint_as_float(v[k]), scale_log2, neg_m));
-          float p1 = ex2(fmaf(__uint_as_float(v[k + 1]), scale_log2, neg_m));
+          const int q = (e >> 1) & 3;
+          float x0, x1, p0, p1;
+          fma2(x0, x1, __uint_as_float(v[k]), __uint_as_float(v[k + 1]), scale_log2, scale_log2, neg_m, neg_m);
+          if (q < kPolyPairs) {
+            exp2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
           if (!full) {
             if (k >= kvalid) p0 = 0.f;
             if (k + 1 >= kvalid) p1 = 0.f;
           }
-          ps[(e >> 1) & 7] += p0 + p1;
+          add2(ps[2 * q], ps[2 * q + 1], ps[2 * q], ps[2 * q + 1], p0, p1);
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st_32x32b_x16(tS + static_cast<uint32_t>(16 * c), pk);
