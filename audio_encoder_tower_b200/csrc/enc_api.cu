@@ -256,21 +256,21 @@ enc_status build(enc_handle* h, const enc_weights* w) {
     ok = ok && make_out_map(&h->m_out_y1, h->y1, (uint64_t)rows_t, (uint64_t)d);
     ok = ok && make_out_map(&h->m_out_qkv, h->qkv, (uint64_t)rows_p, 3 * (uint64_t)d);
     ok = ok && make_out_map(&h->m_out_f, h->f, (uint64_t)rows_p, (uint64_t)F);
-    ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, gemm_tile_n(d));
-    ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, gemm_tile_n(d));
+    ok = ok && map_rows(&h->m_conv1_w, h->conv1_w, 3 * h->mpad, d, 128);
+    ok = ok && map_rows(&h->m_conv2_w, h->conv2_w, 3 * d, d, 128);
     if (ph) {
       ok = ok && map_rows(&h->m_e, h->e, d, rows_o, 128);
       ok = ok && map_rows(&h->m_p1, h->p1, ph, rows_o, 128);
       ok = ok && make_out_map(&h->m_out_p1, h->p1, (uint64_t)rows_o, (uint64_t)ph);
-      ok = ok && map_rows(&h->m_proj1_w, h->proj1_w, d, ph, gemm_tile_n(ph));
-      ok = ok && map_rows(&h->m_proj2_w, h->proj2_w, ph, po, gemm_tile_n(po));
+      ok = ok && map_rows(&h->m_proj1_w, h->proj1_w, d, ph, 128);
+      ok = ok && map_rows(&h->m_proj2_w, h->proj2_w, ph, po, 128);
     }
     h->lmaps.resize(L);
     for (int l = 0; ok && l < L; ++l) {
-      ok = ok && map_rows(&h->lmaps[l].qkv, h->qkv_w[l], d, 3 * d, gemm_tile_n(3 * d));
-      ok = ok && map_rows(&h->lmaps[l].o, h->o_w[l], d, d, gemm_tile_n(d));
-      ok = ok && map_rows(&h->lmaps[l].fc1, h->fc1_w[l], d, F, gemm_tile_n(F));
-      ok = ok && map_rows(&h->lmaps[l].fc2, h->fc2_w[l], F, d, gemm_tile_n(d));
+      ok = ok && map_rows(&h->lmaps[l].qkv, h->qkv_w[l], d, 3 * d, 128);
+      ok = ok && map_rows(&h->lmaps[l].o, h->o_w[l], d, d, 128);
+      ok = ok && map_rows(&h->lmaps[l].fc1, h->fc1_w[l], d, F, 128);
+      ok = ok && map_rows(&h->lmaps[l].fc2, h->fc2_w[l], F, d, 128);
     }
     if (!ok) return ENC_ERR_CUDA;
   }

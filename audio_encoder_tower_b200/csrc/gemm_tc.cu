@@ -167,6 +167,53 @@ __device__ __forceinline__ void epi_store_tile(const EpiParams& e, const CUtenso
   }
 }
 
+// ------------------------------------------------------ pairs of CTAs (2-SM MMA)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory whose transaction bytes count on the
+// barrier of the pair's first CTA (the one that issues the MMAs). Not a
+// multicast: every CTA loads only its own operand halves.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* map, uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256 over the pair.
+__device__ __forceinline__ void umma_f16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` in every CTA of `mask` once the pair's previously issued MMAs are done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
 // Epilogue instantiations: each keeps the whole register budget to itself.
 enum EpiKind : int {
   EK_GENERIC = 0,   // per-thread stores (conv2 scatter + position table, projector scatter)
@@ -223,7 +270,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
           int ax, ay;
           a_coords(p, m0, kb, ax, ay);
           tma_load_2d(sA + stage * C::kABytes, &map_a, &full[stage], ax, ay);
-          tma_load_2d(sB + stage * C::kBBytes, &map_b, &full[stage], kb * BK, n0);
+#pragma unroll
+          for (int half_b = 0; half_b < BN / 128; ++half_b)   // weight maps use 128-row boxes
+            tma_load_2d(sB + stage * C::kBBytes + half_b * (128 * BK * 2), &map_b, &full[stage], kb * BK,
+                        n0 + half_b * 128);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -326,6 +376,197 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pair kernel: a cluster of two CTAs on two SMs computes 256 x 256 output tiles
+// with tcgen05.mma.cta_group::2 (M = 256). CTA r of the pair holds rows
+// 128r .. 128r+127 of the A tile and rows 128r .. 128r+127 of the B tile (half
+// of the tile's columns) in a 6-stage ring of 32 KB per stage; the MMA reads
+// both CTAs' halves. Against the single-CTA kernel each SM loads a third less
+// operand data per MMA and keeps more stages in flight.
+//   warp 0 (both CTAs)  TMA producer for the CTA's own halves; the bytes count
+//                       on the first CTA's stage barrier.
+//   warp 1 (first CTA)  MMA issuer; multicast commits free the stage in both
+//                       CTAs and publish the accumulator to both epilogues.
+//   warps 2..9 (both)   epilogue of the CTA's 128 rows, as in the single-CTA
+//                       kernel; they release the accumulator on the first
+//                       CTA's barrier.
+// ---------------------------------------------------------------------------
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairABytes = 128 * BK * 2;   // this CTA's 128 rows of A
+constexpr uint32_t kPairBBytes = 128 * BK * 2;   // this CTA's 128 rows of B
+constexpr size_t kPairSmemBytes = 1024 + kPairStages * (size_t)(kPairABytes + kPairBBytes) + 1024 +
+                                  (size_t)kEpiWarps * 32 * 32 * 4;
+
+template <int kEpi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const __grid_constant__ CUtensorMap map_c, const GemmTcParams p) {
+  constexpr int BN = 256;
+  constexpr uint32_t kTmemCols = 2 * BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);   // used in the first CTA
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;   // [2]
+  uint64_t* tempty = tfull + 2;            // [2] used in the first CTA
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* stage_c = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 1024);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2 * kEpiWarps * 32); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&map_a); tma_prefetch_desc(&map_b); }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // both CTAs' barriers exist before any remote arrive or transaction
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t armed = 0, armed_phase = 0;
+      for (int tile = cluster; ok && tile < p.num_tiles; tile += nclusters) {
+        const int m0 = (tile / p.tiles_n) * 256 + 128 * static_cast<int>(rank);
+        const int n0 = (tile % p.tiles_n) * BN + 128 * static_cast<int>(rank);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
+          const uint32_t bar = peer_addr(&full[stage], 0);
+          int ax, ay;
+          a_coords(p, m0, kb, ax, ay);
+          tma_load_2d_pair(sA + stage * kPairABytes, &map_a, bar, ax, ay);
+          tma_load_2d_pair(sB + stage * kPairBBytes, &map_b, bar, kb * BK, n0);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        set_status(p.status, kDevTimeout);
+        *abort_v = 1;
+        // the first CTA's barriers track the copies; let them land before leaving
+        if (leader)
+          for (int s = 0; s < kPairStages; ++s)
+            if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      for (int tile = cluster; ok && tile < p.num_tiles; tile += nclusters) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * kPairABytes));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * kPairBBytes));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                             idesc, (kb | k) != 0 ? 1u : 0u);
+          issued = true;
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) { set_status(p.status, kDevTimeout); *abort_v = 1; }
+      if (issued) {   // every MMA done before the pair's TMEM and shared memory go away
+        umma_commit_pair(drain, 0x1);
+        mbar_wait(drain, 0, nullptr, kWaitLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    constexpr int NC = BN / 64;            // 32-column chunks per epilogue warp
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tempty_leader[2] = {peer_addr(&tempty[0], 0), peer_addr(&tempty[1], 0)};
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < p.num_tiles; tile += nclusters) {
+      const int m0 = (tile / p.tiles_n) * 256 + 128 * static_cast<int>(rank);
+      const int n0 = (tile % p.tiles_n) * BN + half * (BN / 2);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
+        set_status(p.status, kDevTimeout);
+        *abort_v = 1;
+        break;
+      }
+      tc_fence_after();
+      const int r = m0 + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      if constexpr (kEpi == EK_RESID) {
+        epi_residual_tile<NC>(p.epi, &map_c, m0 + quarter * 32, n0, taddr, stage_c + (warp - 2) * 32 * 32, lane);
+      } else if constexpr (kEpi == EK_STORE) {
+        epi_store_tile<NC / 2>(p.epi, &map_c, m0 + quarter * 32, n0, taddr,
+                               reinterpret_cast<uint32_t*>(stage_c + (warp - 2) * 32 * 32), lane);
+      } else {
+        int dst = 0, pe_row = 0;
+        bool zero = false;
+        const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+          tmem_wait_ld();
+          if (row_ok)
+            epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if constexpr (kEpi != EK_GENERIC) {
+      if (lane == 0) bulk_wait0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // no CTA leaves while its pair may still read its memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -396,23 +637,59 @@ bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int kEpi>
+cudaError_t launch_pair(const CUtensorMap& map_a, const CUtensorMap& map_b, const CUtensorMap& map_c,
+                        const GemmTcParams& p, int sm_count, cudaStream_t stream) {
+  static unsigned long long done = 0;
+  static int max_clusters[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(done & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sm_count / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<kEpi>, &cfg);
+    if (e != cudaSuccess || n < 1) n = sm_count / 2;   // every SM pairs up
+    cudaGetLastError();
+    max_clusters[dev & 63] = n;
+    done |= bit;
+  }
+  const int clusters = p.num_tiles < max_clusters[dev & 63] ? p.num_tiles : max_clusters[dev & 63];
+  gemm_tc2_kernel<kEpi><<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(map_a, map_b, map_c, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_tc(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
                            cudaStream_t stream, const CUtensorMap* map_c) {
   if (p.M <= 0) return cudaSuccess;
   const int bn = gemm_tile_n(p.N);
-  p.tiles_n = p.N / bn;
-  p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
-  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
   const bool resid = p.epi.mode == EPI_RESIDUAL;
   if (resid && !map_c) return cudaErrorInvalidValue;
   // bf16 row outputs go through TMA stores when the caller supplied the output map
   const bool store = !resid && map_c && (p.epi.mode == EPI_STORE || p.epi.mode == EPI_CONV1);
   const CUtensorMap& mc = map_c ? *map_c : map_a;
-  if (bn == 256) {
-    if (resid) return launch_one<256, EK_RESID>(map_a, map_b, mc, p, grid, stream);
-    if (store) return launch_one<256, EK_STORE>(map_a, map_b, mc, p, grid, stream);
-    return launch_one<256, EK_GENERIC>(map_a, map_b, mc, p, grid, stream);
+  p.tiles_n = p.N / bn;
+  if (bn == 256) {   // 256 x 256 tiles on pairs of SMs
+    p.num_tiles = ((p.M + 255) / 256) * p.tiles_n;
+    if (resid) return launch_pair<EK_RESID>(map_a, map_b, mc, p, sm_count, stream);
+    if (store) return launch_pair<EK_STORE>(map_a, map_b, mc, p, sm_count, stream);
+    return launch_pair<EK_GENERIC>(map_a, map_b, mc, p, sm_count, stream);
   }
+  p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
+  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
   if (resid) return launch_one<128, EK_RESID>(map_a, map_b, mc, p, grid, stream);
   if (store) return launch_one<128, EK_STORE>(map_a, map_b, mc, p, grid, stream);
   return launch_one<128, EK_GENERIC>(map_a, map_b, mc, p, grid, stream);

@@ -30,7 +30,7 @@ enc_status enc_linear_bf16(const void* A, const void* W, const float* bias, void
   if (sms <= 0) return ENC_ERR_CUDA;
   CUtensorMap ma, mb;
   if (!make_tma_2d(&ma, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128)) return ENC_ERR_CUDA;
-  if (!make_tma_2d(&mb, W, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, (uint32_t)gemm_tile_n(N)))
+  if (!make_tma_2d(&mb, W, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, 128))
     return ENC_ERR_CUDA;
   GemmTcParams p;
   memset(&p, 0, sizeof(p));
