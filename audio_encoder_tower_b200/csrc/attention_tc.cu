@@ -11,7 +11,7 @@
 // One CTA = 128 query rows of one (clip, head); two CTAs share an SM, so one
 // CTA's exponentials overlap the other's waits. K/V stream in tiles of 96 keys.
 //   warp 0      TMA: Q once, then K_j and V_j into a 3-stage ring (128-byte swizzle).
-//   warp 1      MMA issuer. S_j = Q K_j^T (M=128, N=96, K=64) goes to score
+//   warp 1      MMA issuer (whole warp, one elected lane). S_j = Q K_j^T (M=128, N=96, K=64) goes to score
 //               buffer j%2, so S_{j+1} is ready while the softmax works on S_j.
 //               O += P_j V_j reads P_j from TMEM (A operand in tensor memory):
 //               the softmax writes P_j (bf16) over the first 48 columns of S_j's
@@ -28,6 +28,8 @@
 // (setmaxnreg): 128*56 + 128*200 = 256*128.
 //
 // TMEM (256 columns per CTA): S0/P0 [0,96), S1/P1 [96,192), O [192,256).
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -68,6 +70,18 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -86,6 +100,15 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// One lane of a converged warp (the lowest active one) for single-thread issue.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
 }
 
 // Packed fp32 pairs (one instruction for two lanes of work on sm_100).
@@ -216,53 +239,83 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         for (int t = armed_upto - kStages; t < armed_upto; ++t)
           if (t >= 0) mbar_wait(&kv_full[slot(t)], fill_parity(t), nullptr, kWaitNs / 4);
       }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // ------------------------------------------------------------ MMA
+      // The whole warp walks the schedule and one elected lane issues, so the
+      // operands stay warp-uniform (a tcgen05.mma issued from divergent code
+      // costs several times more issue cycles). The loop is unrolled by the two
+      // score buffers so their TMEM offsets are constants.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHD) | (1u << 16);   // B (V) MN-major
-      bool ok = mbar_wait(q_full, 0, abort_v, kWaitNs);
-      bool issued = false;
+      constexpr uint64_t kSlotDesc = kKVBytes >> 4;   // one ring slot in descriptor address units
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, kWaitNs));
+      };
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
-      auto issue_s = [&](int j) {   // S_j = Q K_j^T into buffer j % 2
-        const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + slot(j) * kKVBytes));
-        const uint32_t dS = tmem + kColS + static_cast<uint32_t>((j & 1) * kKT);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sK));
+      const uint64_t vdesc0 = smem_desc_sw128_mn(smem_u32(sV));
+      bool issued = false;
+      auto issue_s = [&](int j, auto buf) {   // S_j = Q K_j^T into buffer `buf` (= j % 2)
+        constexpr uint32_t bf = decltype(buf)::value;
+        const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(slot(j)) * kSlotDesc;
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)
-          umma_f16_ss(dS, qdesc + static_cast<uint64_t>(2 * k), kdesc + static_cast<uint64_t>(2 * k), idesc_s,
-                      k > 0 ? 1u : 0u);
-        umma_commit(&s_full[j & 1]);
+          for (int k = 0; k < kHD / 16; ++k)
+            umma_f16_ss(tmem + kColS + bf * kKT, qdesc + static_cast<uint64_t>(2 * k),
+                        kdesc + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
+          umma_commit(&s_full[bf]);
+        }
+        __syncwarp();
         issued = true;
       };
-      for (int j = 0; ok && j < 2 && j < nkv; ++j) {
-        ok = mbar_wait(&kv_full[slot(j)], fill_parity(j), abort_v, kWaitNs);
-        if (ok) { tc_fence_after(); issue_s(j); }
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int bf = j & 1;
+      auto step = [&](int j, auto buf) {   // P_j V_j, then S_{j+2} into the same buffer
+        constexpr uint32_t bf = decltype(buf)::value;
         const uint32_t use = static_cast<uint32_t>((j >> 1) & 1);
-        if (!mbar_wait(&p_full[bf], use, abort_v, kWaitNs)) { ok = false; break; }
+        if (!wait_all(&p_full[bf], use)) return false;
         tc_fence_after();
         // O += P_j V_j: P_j in the first 48 columns of buffer j % 2, 16 keys (8 columns) per step
-        const uint64_t vdesc = smem_desc_sw128_mn(smem_u32(sV + slot(j) * kKVBytes));
-        const uint32_t aP = tmem + kColS + static_cast<uint32_t>(bf * kKT);
+        const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(slot(j)) * kSlotDesc;
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < kKT / 16; ++k)
-          umma_f16_ts(tmem + kColO, aP + static_cast<uint32_t>(8 * k), vdesc + static_cast<uint64_t>(128 * k),
-                      idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&pv_done[bf]);
-        umma_commit(&kv_empty[slot(j)]);
+          for (int k = 0; k < kKT / 16; ++k)
+            umma_f16_ts(tmem + kColO, tmem + kColS + bf * kKT + static_cast<uint32_t>(8 * k),
+                        vdesc + static_cast<uint64_t>(128 * k), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&pv_done[bf]);
+          umma_commit(&kv_empty[slot(j)]);
+        }
+        __syncwarp();
         if (j + 2 < nkv) {
           // S_{j+2} overwrites buffer j % 2: P_j V_j must have read P_j first
-          if (!mbar_wait(&pv_done[bf], use, abort_v, kWaitNs)) { ok = false; break; }
-          if (!mbar_wait(&kv_full[slot(j + 2)], fill_parity(j + 2), abort_v, kWaitNs)) { ok = false; break; }
+          if (!wait_all(&pv_done[bf], use)) return false;
+          if (!wait_all(&kv_full[slot(j + 2)], fill_parity(j + 2))) return false;
           tc_fence_after();
-          issue_s(j + 2);
+          issue_s(j + 2, buf);
+        }
+        return true;
+      };
+      using Buf0 = std::integral_constant<uint32_t, 0>;
+      using Buf1 = std::integral_constant<uint32_t, 1>;
+      bool ok = wait_all(q_full, 0) && wait_all(&kv_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, Buf0{});
+      }
+      if (ok && nkv > 1) {
+        ok = wait_all(&kv_full[1], 0);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1, Buf1{});
         }
       }
-      if (!ok) { set_status(status, kDevTimeout); *abort_v = 1; }
+      for (int j = 0; ok && j < nkv; j += 2) {
+        ok = step(j, Buf0{});
+        if (ok && j + 1 < nkv) ok = step(j + 1, Buf1{});
+      }
+      if (!ok && lane == 0) { set_status(status, kDevTimeout); *abort_v = 1; }
       if (issued) {   // every MMA done: O final, TMEM safe to release
-        umma_commit(o_done);
-        mbar_wait(o_done, 0, nullptr, kWaitNs);
+        if (elect_one()) umma_commit(o_done);
+        __syncwarp();
+        wait_all(o_done, 0);
       }
     }
   } else {
@@ -354,14 +407,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < kHD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tO + static_cast<uint32_t>(32 * c), o);
+        // 8 columns at a time: the whole score row is still held in registers
+#pragma unroll 1
+        for (int c = 0; c < kHD / 8; ++c) {
+          uint32_t o[8];
+          tmem_ld_32x32b_x8(tO + static_cast<uint32_t>(8 * c), o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st_32x32b_x32(tO + static_cast<uint32_t>(32 * c), o);
+          for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st_32x32b_x8(tO + static_cast<uint32_t>(8 * c), o);
         }
       }
       tmem_wait_st();
