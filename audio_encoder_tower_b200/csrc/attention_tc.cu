@@ -102,15 +102,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// One lane of a converged warp (the lowest active one) for single-thread issue.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t p;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\telect.sync R|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(p));
-  return p != 0;
-}
-
 // Packed fp32 pairs (one instruction for two lanes of work on sm_100).
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
                                      float c1) {
@@ -248,9 +239,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHD) | (1u << 16);   // B (V) MN-major
       constexpr uint64_t kSlotDesc = kKVBytes >> 4;   // one ring slot in descriptor address units
-      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, kWaitNs));
-      };
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) { return mbar_wait_warp(bar, parity, abort_v, kWaitNs); };
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sK));
       const uint64_t vdesc0 = smem_desc_sw128_mn(smem_u32(sV));

@@ -289,38 +289,44 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true, issued = false;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+    // The whole warp walks the schedule and one elected lane issues and commits.
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+    const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA)), bdesc0 = smem_desc_sw128(smem_u32(sB));
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true, issued = false;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait_warp(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * C::kABytes));
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * C::kBBytes));
+        // descriptor start addresses advance in 16-byte units
+        const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage) * (C::kABytes >> 4);
+        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(stage) * (C::kBBytes >> 4);
+        if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K inside the swizzled row
             umma_f16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k), idesc,
                         (kb | k) != 0 ? 1u : 0u);
-          issued = true;
           umma_commit(&empty[stage]);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        __syncwarp();
+        issued = true;
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) { set_status(p.status, kDevTimeout); *abort_v = 1; }
-      if (issued) {   // every MMA done before TMEM is released
-        umma_commit(drain);
-        mbar_wait(drain, 0, nullptr, kWaitLimitNs);
-      }
+      if (!ok) break;
+      if (elect_one()) umma_commit(&tfull[acc]);
+      __syncwarp();
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (!ok && lane == 0) { set_status(p.status, kDevTimeout); *abort_v = 1; }
+    if (issued) {   // every MMA done before TMEM is released
+      if (elect_one()) umma_commit(drain);
+      __syncwarp();
+      mbar_wait_warp(drain, 0, nullptr, kWaitLimitNs);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -476,37 +482,44 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (leader && lane == 0) {
+    // first CTA only: the whole warp walks the schedule, one elected lane issues
+    if (leader) {
       constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA)), bdesc0 = smem_desc_sw128(smem_u32(sB));
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
       for (int tile = cluster; ok && tile < p.num_tiles; tile += nclusters) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait_warp(&full[stage], phase, abort_v, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * kPairABytes));
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * kPairBBytes));
+          const uint64_t adesc = adesc0 + static_cast<uint64_t>(stage) * (kPairABytes >> 4);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(stage) * (kPairBBytes >> 4);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_f16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
-                             idesc, (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16_ss_pair(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                               idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_commit_pair(&empty[stage], 0x3);
+          }
+          __syncwarp();
           issued = true;
-          umma_commit_pair(&empty[stage], 0x3);
           if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit_pair(&tfull[acc], 0x3);
+        if (elect_one()) umma_commit_pair(&tfull[acc], 0x3);
+        __syncwarp();
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) { set_status(p.status, kDevTimeout); *abort_v = 1; }
+      if (!ok && lane == 0) { set_status(p.status, kDevTimeout); *abort_v = 1; }
       if (issued) {   // every MMA done before the pair's TMEM and shared memory go away
-        umma_commit_pair(drain, 0x1);
-        mbar_wait(drain, 0, nullptr, kWaitLimitNs);
+        if (elect_one()) umma_commit_pair(drain, 0x1);
+        __syncwarp();
+        mbar_wait_warp(drain, 0, nullptr, kWaitLimitNs);
       }
     }
   } else {
