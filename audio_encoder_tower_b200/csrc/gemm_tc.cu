@@ -144,17 +144,26 @@ __device__ __forceinline__ void epi_store_tile(const EpiParams& e, const CUtenso
     if (lane == 0) bulk_wait_read0();   // the previous store has read the staging tile
     tmem_wait_ld();
     __syncwarp();
-    const float* bias = e.bias ? e.bias + n0 + c * 64 : nullptr;
+    const float4* bias = e.bias ? reinterpret_cast<const float4*>(e.bias + n0 + c * 64) : nullptr;
     uint4* row = reinterpret_cast<uint4*>(tile + lane * 32);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {   // 8 columns -> one 16-byte piece
       float t[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float a = __uint_as_float(v[8 * j + i]) + (bias ? bias[8 * j + i] : 0.f);
-        a = g ? gelu_fast(a) : a;
-        t[i] = zero ? 0.f : a;
+      for (int i = 0; i < 8; ++i) t[i] = __uint_as_float(v[8 * j + i]);
+      if (bias) {   // the same 32 bytes for every lane: one broadcast load
+        const float4 b0 = __ldg(bias + 2 * j), b1 = __ldg(bias + 2 * j + 1);
+        add2(t[0], t[1], t[0], t[1], b0.x, b0.y);
+        add2(t[2], t[3], t[2], t[3], b0.z, b0.w);
+        add2(t[4], t[5], t[4], t[5], b1.x, b1.y);
+        add2(t[6], t[7], t[6], t[7], b1.z, b1.w);
       }
+      if (g) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) gelu_fast2(t[i], t[i + 1]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t[i] = zero ? 0.f : t[i];
       row[j ^ (lane & 7)] = make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]), pack_bf16x2(t[4], t[5]),
                                        pack_bf16x2(t[6], t[7]));
     }

@@ -19,8 +19,10 @@ def _dev(a, dtype=None):
     return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype or torch.bfloat16)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (127, 256, 128), (128, 384, 64), (300, 1280, 1280),
-                                   (1000, 512, 320), (4000, 3840, 1280)])
+# N % 256 == 0 runs 256 x 256 tiles on pairs of SMs: M = 129 leaves the second
+# CTA of the pair one valid row, M = 257 starts a second tile row
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (127, 256, 128), (128, 384, 64), (129, 256, 64), (257, 512, 64),
+                                   (300, 1280, 1280), (1000, 512, 320), (4000, 3840, 1280)])
 @pytest.mark.parametrize("gelu", [False, True])
 def test_linear_bf16(M, N, K, gelu):
     import torch
@@ -38,7 +40,8 @@ def test_linear_bf16(M, N, K, gelu):
     assert np.all(err <= 8e-3 * np.maximum(1.0, np.abs(ref))), float(err.max())
 
 
-@pytest.mark.parametrize("M,N,K", [(77, 256, 64), (513, 1280, 5120)])
+# reduce-add epilogue on pairs of SMs: a ragged second tile row (129) and a long K (5120)
+@pytest.mark.parametrize("M,N,K", [(77, 256, 64), (129, 512, 512), (513, 1280, 5120)])
 def test_linear_residual(M, N, K):
     import torch
     from audio_encoder_tower_b200.binding import linear_bf16
