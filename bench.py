@@ -7,6 +7,7 @@ batch 16 per GPU, bf16 operands with fp32 accumulation, synthetic seeded inputs
 and random weights of that architecture.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+    python bench.py --kernel qkv|out|fc1|fc2|attention [--steps K] [--warmup W]   (one kernel alone)
 
 One step = one enc_forward over a batch of 16 clips. Multi-GPU (torchrun, one
 process per GPU) runs independent replicas, each with its own batch of 16
@@ -209,6 +210,47 @@ def gemm_traffic_record():
     return rec if rec.get("source_sha256") == h.hexdigest() else None
 
 
+# ------------------------------------------------------- one kernel alone
+def run_kernel(args, cfg):
+    """Time one layer kernel of the workload alone through the C ABI (for profiling):
+    a layer GEMM shape (qkv, out, fc1, fc2) at M = batch x positions, or the attention."""
+    import torch
+    from audio_encoder_tower_b200.binding import attention_bf16, linear_bf16
+    torch.cuda.set_device(0)
+    n = cfg.frames // 2
+    M, d, f, H = cfg.batch * n, cfg.d_model, cfg.ffn_dim, cfg.n_heads
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed)
+    if args.kernel == "attention":
+        qkv = torch.randn(M, 3 * d, device="cuda", generator=g).to(torch.bfloat16)
+        out = torch.empty(M, d, device="cuda", dtype=torch.bfloat16)
+        cu = torch.arange(0, (cfg.batch + 1) * n, n, device="cuda", dtype=torch.int32)
+        launch = lambda: attention_bf16(qkv, cu, n, H, out=out)   # noqa: E731
+        flops = 4.0 * cfg.batch * n * n * d
+        shape = {"clips": cfg.batch, "positions": n, "heads": H, "head_dim": 64}
+    else:
+        N, K, gelu, resid = {"qkv": (3 * d, d, False, False), "out": (d, d, False, True),
+                             "fc1": (f, d, True, False), "fc2": (d, f, False, True)}[args.kernel]
+        A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, device="cuda", generator=g) * 0.03).to(torch.bfloat16)
+        b = torch.randn(N, device="cuda", generator=g) * 0.1
+        x = torch.zeros(M, N, device="cuda", dtype=torch.float32) if resid else None
+        launch = lambda: linear_bf16(A, W, b, gelu=gelu, resid=x)   # noqa: E731
+        flops = 2.0 * M * N * K
+        shape = {"M": M, "N": N, "K": K, "gelu": gelu, "residual": resid}
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        launch()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"kernel": args.kernel, "workload": cfg.name, "shape": shape, "launches": args.steps,
+                      "ms_per_launch": ms, "tflops": flops / ms / 1e9}), flush=True)
+
+
 # ---------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -218,9 +260,13 @@ def main():
     ap.add_argument("--config", default="large_b16", choices=S.CONFIG_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention"],
+                    help="time one layer kernel of the workload alone (profiling aid)")
     args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
     cfg = S.CONFIGS[args.config]
+    if args.kernel:
+        return run_kernel(args, cfg)
+    args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
