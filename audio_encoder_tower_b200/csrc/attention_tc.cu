@@ -133,6 +133,39 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr) {
   return d;
 }
 
+// P = exp2(s * scale_log2 - m) for one 96-key score row (this thread's TMEM
+// lane), written as bf16 pairs over the row's first 48 columns, 32 keys at a
+// time; row sums into ps. kMasked zeroes keys >= kvalid (the clip's last key
+// tile only, so full tiles carry no compare-and-select per key).
+template <bool kMasked>
+__device__ __forceinline__ void softmax_exps(const uint32_t (&v)[kKT], uint32_t tS, float scale_log2, float neg_m,
+                                             int kvalid, float (&ps)[8]) {
+#pragma unroll
+  for (int c = 0; c < kKT / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int k = 32 * c + e;
+      const int q = (e >> 1) & 3;
+      float x0, x1, p0, p1;
+      fma2(x0, x1, __uint_as_float(v[k]), __uint_as_float(v[k + 1]), scale_log2, scale_log2, neg_m, neg_m);
+      if (q < kPolyPairs) {
+        exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      if constexpr (kMasked) {
+        if (k >= kvalid) p0 = 0.f;
+        if (k + 1 >= kvalid) p1 = 0.f;
+      }
+      add2(ps[2 * q], ps[2 * q + 1], ps[2 * q], ps[2 * q + 1], p0, p1);
+      pk[e >> 1] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_32x32b_x16(tS + static_cast<uint32_t>(16 * c), pk);
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -337,35 +370,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
           l_run *= alpha;
         }
       }
-      // P = exp2(s * scale_log2 - m) (0 on masked keys) as bf16 pairs over the
-      // first 48 columns of this score buffer, 32 keys at a time
-      const float neg_m = -m_run;
+      // P = exp2(s * scale_log2 - m) as bf16 pairs over the first 48 columns of
+      // this score buffer; only the clip's last key tile takes the masked copy
       float ps[8];   // eight independent partial row sums (four packed pairs)
 #pragma unroll
       for (int q = 0; q < 8; ++q) ps[q] = 0.f;
-#pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int k = 32 * c + e;
-          const int q = (e >> 1) & 3;
-          float x0, x1, p0, p1;
-          fma2(x0, x1, __uint_as_float(v[k]), __uint_as_float(v[k + 1]), scale_log2, scale_log2, neg_m, neg_m);
-          if (q < kPolyPairs) {
-            exp2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          if (!full) {
-            if (k >= kvalid) p0 = 0.f;
-            if (k + 1 >= kvalid) p1 = 0.f;
-          }
-          add2(ps[2 * q], ps[2 * q + 1], ps[2 * q], ps[2 * q + 1], p0, p1);
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st_32x32b_x16(tS + static_cast<uint32_t>(16 * c), pk);
+      if (full) {
+        softmax_exps<false>(v, tS, scale_log2, -m_run, kvalid, ps);
+      } else {
+        softmax_exps<true>(v, tS, scale_log2, -m_run, kvalid, ps);
       }
       l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       if (rescale) {   // O must hold P_{j-1} V_{j-1} before it is scaled
