@@ -21,7 +21,8 @@ ENC_DTYPE_BF16, ENC_DTYPE_FP32 = 0, 1
 
 EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status", "enc_destroy",
             "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
-            "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch"]
+            "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch",
+            "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy"]
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -98,6 +99,12 @@ def load_library(path: str = LIB_PATH):
     lib.enc_launch_count.restype = ctypes.c_int64
     lib.enc_forward_static_scratch.argtypes = [_VP, _VP, i32p, ctypes.c_int32, _VP, _VP]
     lib.enc_forward_static_scratch.restype = ctypes.c_int
+    lib.enc_frontend_create.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p)]
+    lib.enc_frontend_create.restype = ctypes.c_int
+    lib.enc_frontend_log_mel.argtypes = [_VP, _VP, ctypes.c_int32, _VP, ctypes.c_int32, _VP]
+    lib.enc_frontend_log_mel.restype = ctypes.c_int
+    lib.enc_frontend_destroy.argtypes = [_VP]
+    lib.enc_frontend_destroy.restype = None
     _LIB = lib
     return lib
 
@@ -263,3 +270,39 @@ def attention_bf16(qkv, cu, max_n, n_heads, out=None, status=None, stream=None):
                                              int(max_n), int(n_heads), _ptr(status), _stream_handle(stream)),
            "enc_attention_bf16")
     return out
+
+
+class Frontend:
+    """Log-mel front end (enc_frontend_create / enc_frontend_log_mel / enc_frontend_destroy):
+    30 s clips of 16 kHz audio, fp32 [B, 480000] on the device -> [B, n_mels, 3000]."""
+
+    SAMPLES, FRAMES = 480000, 3000
+
+    def __init__(self, n_mels: int = 128, max_batch: int = 16):
+        self.lib = load_library()
+        h = ctypes.c_void_p()
+        _check(self.lib.enc_frontend_create(int(n_mels), int(max_batch), ctypes.byref(h)), "enc_frontend_create")
+        self.h, self.n_mels, self.max_batch = h, int(n_mels), int(max_batch)
+
+    def log_mel(self, audio, out=None, dtype="bf16", stream=None):
+        import torch
+        B = audio.shape[0]
+        if audio.dtype != torch.float32 or tuple(audio.shape[1:]) != (self.SAMPLES,) or not audio.is_contiguous():
+            raise ValueError("audio must be a contiguous fp32 [B, 480000] device tensor")
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        if out is None:
+            out = torch.empty((B, self.n_mels, self.FRAMES), dtype=tdt, device=audio.device)
+        _check(self.lib.enc_frontend_log_mel(self.h, _ptr(audio), int(B), _ptr(out), 0 if dtype == "bf16" else 1,
+                                             _stream_handle(stream)), "enc_frontend_log_mel")
+        return out
+
+    def close(self):
+        if self.h:
+            self.lib.enc_frontend_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,260 @@
+// Log-mel front end on the GPU (fp32, CUDA cores): 30 s of 16 kHz audio ->
+// the encoder's [n_mels, 3000] input features. Geometry from the pages
+// (Voxtral-Mini-3B-2507, "Preprocessor": WhisperFeatureExtractor, 480,000
+// samples, hop 160, 3000 frames, 128 features; MiniCPM-o-2.6, "(2) AUDIO": 80);
+// window, filterbank and compression as the Whisper feature extractor
+// (include/enc_frontend.h lists them).
+//
+// Steps for B clips:
+//   1. pad_kernel: each clip reflected by 200 samples at both ends into rows of
+//      a buffer whose clip stride is 3003 frames x 160 samples, so frame f of
+//      clip b starts at sample (b * 3003 + f) * 160 for every clip
+//   2. SGEMM: overlapping 400-sample rows (row stride 160) x the windowed
+//      cos / sin basis -> X [B * 3003, 404] (real | imaginary parts)
+//   3. power_kernel: |X_k|^2 for the 201 bins
+//   4. SGEMM: power x filterbank^T -> mel [B * 3003, n_mels]
+//   5. log_max_kernel: log10(max(mel, 1e-10)) in place over the 3000 frames
+//      kept, and the clip's maximum
+//   6. finish_kernel: max(x, clip max - 8), (x + 4) / 4, transposed to
+//      [B, n_mels, 3000]
+// Rows 3000..3002 of every clip are computed and dropped (they keep the frame
+// stride uniform across clips).
+#include <cmath>
+#include <cstdlib>
+#include <new>
+#include <vector>
+
+#include "../../include/enc_frontend.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace enc {
+namespace {
+
+constexpr int kSamples = 480000, kFft = 400, kHop = 160, kFrames = 3000;
+constexpr int kBins = kFft / 2 + 1;               // 201
+constexpr int kFramesPad = kSamples / kHop + 3;   // 3003 frame rows per clip
+constexpr int kClipStride = kFramesPad * kHop;    // 480,480 padded samples per clip
+constexpr int kBasisRows = 404;                   // cos k = 0..200, sin k = 0..200, two zero rows
+constexpr int kPowCols = 204;                     // 201 bins + 3 zero columns
+constexpr int kSlack = 512;                       // read past the last clip by its dropped frame rows
+static_assert((kFramesPad - 1) * kHop + kFft <= kClipStride + kSlack, "slack covers the dropped rows");
+
+__global__ void pad_kernel(const float* __restrict__ audio, float* __restrict__ padded, int B) {
+  const size_t total = static_cast<size_t>(B) * kClipStride;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(i / kClipStride);
+    int s = static_cast<int>(i - static_cast<size_t>(b) * kClipStride) - kFft / 2;
+    if (s < 0) s = -s;                                    // reflect, edge sample not repeated
+    if (s >= kSamples) s = 2 * (kSamples - 1) - s;
+    padded[i] = audio[static_cast<size_t>(b) * kSamples + s];
+  }
+}
+
+__global__ void power_kernel(const float* __restrict__ X, float* __restrict__ P, int rows) {
+  const size_t total = static_cast<size_t>(rows) * kPowCols;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = i / kPowCols;
+    const int k = static_cast<int>(i - r * kPowCols);
+    float p = 0.f;
+    if (k < kBins) {
+      const float re = X[r * kBasisRows + k], im = X[r * kBasisRows + kBins + k];
+      p = fmaf(re, re, im * im);
+    }
+    P[i] = p;
+  }
+}
+
+// fp32 keys whose unsigned order is the float order (for atomicMax)
+__device__ __forceinline__ unsigned order_key(float x) {
+  const unsigned u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_order_key(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// grid (ceil(3000 * n_mels / 256 / 8), B): 8 values per thread
+__global__ void log_max_kernel(float* __restrict__ M, int n_mels, unsigned* __restrict__ cmax) {
+  const int b = blockIdx.y;
+  float* m = M + static_cast<size_t>(b) * kFramesPad * n_mels;   // the clip's frame-major rows
+  const int count = kFrames * n_mels;
+  float best = -INFINITY;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) {
+    const float v = log10f(fmaxf(m[i], 1e-10f));
+    m[i] = v;
+    best = fmaxf(best, v);
+  }
+  best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
+  best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
+  best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 4));
+  best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 2));
+  best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 1));
+  if ((threadIdx.x & 31) == 0 && best > -INFINITY) atomicMax(&cmax[b], order_key(best));
+}
+
+// 32 frames x 32 mel channels per block, transposed through shared memory
+template <typename OutT>
+__global__ void finish_kernel(const float* __restrict__ L, const unsigned* __restrict__ cmax, OutT* __restrict__ mel,
+                              int n_mels) {
+  __shared__ float tile[32][33];
+  const int b = blockIdx.z, f0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
+  const float floor_v = from_order_key(cmax[b]) - 8.0f;
+  const float* src = L + static_cast<size_t>(b) * kFramesPad * n_mels;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int f = f0 + i, m = m0 + threadIdx.x;
+    tile[i][threadIdx.x] = (f < kFrames && m < n_mels) ? src[static_cast<size_t>(f) * n_mels + m] : 0.f;
+  }
+  __syncthreads();
+  OutT* dst = mel + static_cast<size_t>(b) * n_mels * kFrames;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int m = m0 + i, f = f0 + threadIdx.x;
+    if (m < n_mels && f < kFrames)
+      dst[static_cast<size_t>(m) * kFrames + f] = from_float<OutT>((fmaxf(tile[threadIdx.x][i], floor_v) + 4.0f) * 0.25f);
+  }
+}
+
+// ------------------------------------------------------------ host constants
+// Windowed DFT basis: row k = w[n] cos(2 pi k n / 400), row 201 + k = w[n] sin(2 pi k n / 400),
+// w the periodic Hann window; angles reduced exactly ((k n) mod 400) and evaluated in double.
+std::vector<float> dft_basis() {
+  std::vector<float> basis(static_cast<size_t>(kBasisRows) * kFft, 0.f);
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int k = 0; k < kBins; ++k)
+    for (int n = 0; n < kFft; ++n) {
+      const double w = 0.5 - 0.5 * std::cos(two_pi * n / kFft);
+      const double a = two_pi * static_cast<double>((k * n) % kFft) / kFft;
+      basis[static_cast<size_t>(k) * kFft + n] = static_cast<float>(w * std::cos(a));
+      basis[static_cast<size_t>(kBins + k) * kFft + n] = static_cast<float>(w * std::sin(a));
+    }
+  return basis;
+}
+
+// Slaney mel scale: 3 mels per 200 Hz up to 1 kHz, then 27 mels per factor 6.4.
+double slaney_mel(double hz) {
+  return hz < 1000.0 ? hz * 3.0 / 200.0 : 15.0 + std::log(hz / 1000.0) * 27.0 / std::log(6.4);
+}
+double slaney_hz(double mel) {
+  return mel < 15.0 ? mel * 200.0 / 3.0 : 1000.0 * std::exp((mel - 15.0) * std::log(6.4) / 27.0);
+}
+
+// [n_mels, kPowCols]: triangles between n_mels + 2 mel-spaced points from 0 Hz to 8 kHz,
+// on bin frequencies k * 40 Hz, each scaled to unit area (2 / (upper - lower edge)).
+std::vector<float> mel_bank(int n_mels) {
+  std::vector<double> edge(n_mels + 2);
+  const double top = slaney_mel(8000.0);
+  for (int i = 0; i < n_mels + 2; ++i) edge[i] = slaney_hz(top * i / (n_mels + 1));
+  std::vector<float> fb(static_cast<size_t>(n_mels) * kPowCols, 0.f);
+  for (int m = 0; m < n_mels; ++m)
+    for (int k = 0; k < kBins; ++k) {
+      const double f = 40.0 * k;
+      const double rise = (f - edge[m]) / (edge[m + 1] - edge[m]);
+      const double fall = (edge[m + 2] - f) / (edge[m + 2] - edge[m + 1]);
+      const double t = std::fmax(0.0, std::fmin(rise, fall));
+      fb[static_cast<size_t>(m) * kPowCols + k] = static_cast<float>(t * 2.0 / (edge[m + 2] - edge[m]));
+    }
+  return fb;
+}
+
+EpiParams store_epi(float* out, int ldo) {
+  EpiParams e = {};
+  e.mode = EPI_STORE;
+  e.out = out;
+  e.ldo = ldo;
+  return e;
+}
+
+}  // namespace
+}  // namespace enc
+
+struct enc_frontend {
+  int n_mels = 0, max_batch = 0, device = 0;
+  float *basis = nullptr, *fb = nullptr, *padded = nullptr, *X = nullptr, *P = nullptr, *M = nullptr;
+  unsigned* cmax = nullptr;
+};
+
+extern "C" {
+
+ENC_API void enc_frontend_destroy(enc_frontend* h) {
+  if (!h) return;
+  int prev = 0;
+  const bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+  cudaSetDevice(h->device);
+  for (void* p : {static_cast<void*>(h->basis), static_cast<void*>(h->fb), static_cast<void*>(h->padded),
+                  static_cast<void*>(h->X), static_cast<void*>(h->P), static_cast<void*>(h->M),
+                  static_cast<void*>(h->cmax)})
+    if (p) cudaFree(p);
+  if (have_prev) cudaSetDevice(prev);
+  delete h;
+}
+
+ENC_API enc_status enc_frontend_create(int32_t n_mels, int32_t max_batch, enc_frontend** out) {
+  using namespace enc;
+  if (!out) return ENC_ERR_INVALID_ARG;
+  *out = nullptr;
+  if ((n_mels != 80 && n_mels != 128) || max_batch < 1 || max_batch > 4096) return ENC_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ENC_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ENC_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return ENC_ERR_UNSUPPORTED;
+  enc_frontend* h = new (std::nothrow) enc_frontend;
+  if (!h) return ENC_ERR_OOM;
+  h->n_mels = n_mels;
+  h->max_batch = max_batch;
+  h->device = dev;
+  const size_t rows = static_cast<size_t>(max_batch) * kFramesPad;
+  const size_t padded_n = static_cast<size_t>(max_batch) * kClipStride + kSlack;
+  bool ok = cudaMalloc(&h->basis, sizeof(float) * kBasisRows * kFft) == cudaSuccess &&
+            cudaMalloc(&h->fb, sizeof(float) * n_mels * kPowCols) == cudaSuccess &&
+            cudaMalloc(&h->padded, sizeof(float) * padded_n) == cudaSuccess &&
+            cudaMalloc(&h->X, sizeof(float) * rows * kBasisRows) == cudaSuccess &&
+            cudaMalloc(&h->P, sizeof(float) * rows * kPowCols) == cudaSuccess &&
+            cudaMalloc(&h->M, sizeof(float) * rows * n_mels) == cudaSuccess &&
+            cudaMalloc(&h->cmax, sizeof(unsigned) * max_batch) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    enc_frontend_destroy(h);
+    return ENC_ERR_OOM;
+  }
+  const std::vector<float> basis = dft_basis(), fb = mel_bank(n_mels);
+  ok = cudaMemcpy(h->basis, basis.data(), sizeof(float) * basis.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+       cudaMemcpy(h->fb, fb.data(), sizeof(float) * fb.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+       cudaMemset(h->padded, 0, sizeof(float) * padded_n) == cudaSuccess;   // the slack stays zero
+  if (!ok) {
+    enc_frontend_destroy(h);
+    return ENC_ERR_CUDA;
+  }
+  *out = h;
+  return ENC_OK;
+}
+
+ENC_API enc_status enc_frontend_log_mel(enc_frontend* h, const float* audio, int32_t B, void* mel,
+                                        enc_dtype out_dtype, cudaStream_t stream) {
+  using namespace enc;
+  if (!h || !audio || !mel || B < 1 || B > h->max_batch) return ENC_ERR_INVALID_ARG;
+  if (out_dtype != ENC_DTYPE_BF16 && out_dtype != ENC_DTYPE_FP32) return ENC_ERR_INVALID_ARG;
+  const int rows = B * kFramesPad, nm = h->n_mels;
+  cudaError_t e = cudaSuccess;
+  auto ok = [&](cudaError_t r) { if (e == cudaSuccess) e = r; return e == cudaSuccess; };
+  pad_kernel<<<4 * 148, 256, 0, stream>>>(audio, h->padded, B);
+  ok(cudaGetLastError());
+  ok(launch_sgemm(h->padded, kHop, h->basis, kFft, rows, kBasisRows, kFft, store_epi(h->X, kBasisRows), stream));
+  power_kernel<<<4 * 148, 256, 0, stream>>>(h->X, h->P, rows);
+  ok(cudaGetLastError());
+  ok(launch_sgemm(h->P, kPowCols, h->fb, kPowCols, rows, nm, kPowCols, store_epi(h->M, nm), stream));
+  ok(cudaMemsetAsync(h->cmax, 0, sizeof(unsigned) * B, stream));
+  log_max_kernel<<<dim3(64, B), 256, 0, stream>>>(h->M, nm, h->cmax);
+  ok(cudaGetLastError());
+  const dim3 grid((kFrames + 31) / 32, (nm + 31) / 32, B), block(32, 8);
+  if (out_dtype == ENC_DTYPE_BF16)
+    finish_kernel<bf16><<<grid, block, 0, stream>>>(h->M, h->cmax, static_cast<bf16*>(mel), nm);
+  else
+    finish_kernel<float><<<grid, block, 0, stream>>>(h->M, h->cmax, static_cast<float*>(mel), nm);
+  ok(cudaGetLastError());
+  return e == cudaSuccess ? ENC_OK : ENC_ERR_CUDA;
+}
+
+}  // extern "C"

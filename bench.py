@@ -7,7 +7,7 @@ batch 16 per GPU, bf16 operands with fp32 accumulation, synthetic seeded inputs
 and random weights of that architecture.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-    python bench.py --kernel qkv|out|fc1|fc2|attention [--steps K] [--warmup W]   (one kernel alone)
+    python bench.py --kernel qkv|out|fc1|fc2|attention|frontend [--steps K] [--warmup W]   (one step alone)
 
 One step = one enc_forward over a batch of 16 clips. Multi-GPU (torchrun, one
 process per GPU) runs independent replicas, each with its own batch of 16
@@ -212,15 +212,26 @@ def gemm_traffic_record():
 
 # ------------------------------------------------------- one kernel alone
 def run_kernel(args, cfg):
-    """Time one layer kernel of the workload alone through the C ABI (for profiling):
-    a layer GEMM shape (qkv, out, fc1, fc2) at M = batch x positions, or the attention."""
+    """Time one step of the workload alone through the C ABI (for profiling): a
+    layer GEMM shape (qkv, out, fc1, fc2) at M = batch x positions, the
+    attention, or the log-mel front end over the batch's 30 s clips."""
     import torch
     from audio_encoder_tower_b200.binding import attention_bf16, linear_bf16
     torch.cuda.set_device(0)
     n = cfg.frames // 2
     M, d, f, H = cfg.batch * n, cfg.d_model, cfg.ffn_dim, cfg.n_heads
     g = torch.Generator(device="cuda").manual_seed(cfg.seed)
-    if args.kernel == "attention":
+    if args.kernel == "frontend":
+        from audio_encoder_tower_b200 import Frontend
+        fe = Frontend(n_mels=cfg.n_mels, max_batch=cfg.batch)
+        audio = torch.from_numpy(S.make_audio(cfg.batch)).cuda()
+        mel_out = torch.empty((cfg.batch, cfg.n_mels, 3000), dtype=torch.bfloat16, device="cuda")
+        launch = lambda: fe.log_mel(audio, out=mel_out)   # noqa: E731
+        rows = cfg.batch * 3003   # frame rows as computed (3000 kept per clip)
+        flops = 2.0 * rows * 404 * 400 + 2.0 * rows * cfg.n_mels * 204   # the two fp32 GEMMs as executed
+        shape = {"clips": cfg.batch, "samples": 480000, "n_mels": cfg.n_mels, "frames": 3000,
+                 "audio_s": 30.0 * cfg.batch}
+    elif args.kernel == "attention":
         qkv = torch.randn(M, 3 * d, device="cuda", generator=g).to(torch.bfloat16)
         out = torch.empty(M, d, device="cuda", dtype=torch.bfloat16)
         cu = torch.arange(0, (cfg.batch + 1) * n, n, device="cuda", dtype=torch.int32)
@@ -247,8 +258,11 @@ def run_kernel(args, cfg):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    print(json.dumps({"kernel": args.kernel, "workload": cfg.name, "shape": shape, "launches": args.steps,
-                      "ms_per_launch": ms, "tflops": flops / ms / 1e9}), flush=True)
+    line = {"kernel": args.kernel, "workload": cfg.name, "shape": shape, "launches": args.steps,
+            "ms_per_launch": ms, "tflops": flops / ms / 1e9}
+    if args.kernel == "frontend":
+        line["audio_s_per_s"] = shape["audio_s"] / (ms / 1e3)
+    print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- our arm
@@ -260,7 +274,7 @@ def main():
     ap.add_argument("--config", default="large_b16", choices=S.CONFIG_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention"],
+    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention", "frontend"],
                     help="time one layer kernel of the workload alone (profiling aid)")
     args = ap.parse_args()
     cfg = S.CONFIGS[args.config]

@@ -236,3 +236,23 @@ def mel_clip(cfg: EncoderConfig, b: int) -> np.ndarray:
     n = cfg.n_mels * cfg.frames
     u = uniform_f32(cfg.seed, input_index(cfg), n, 3.0, -1.5, start=b * n)
     return _store(cfg, u).reshape(cfg.n_mels, cfg.frames)
+
+
+def make_audio(batch: int, seed: int = 5) -> np.ndarray:
+    """[batch, 480000] float32 test audio (30 s at 16 kHz) for the log-mel front
+    end: white noise (std 0.05) under a piecewise-constant envelope of 0.5 s
+    segments, one sine tone per clip (100 Hz .. 7.1 kHz, amplitude 0.05 .. 0.35),
+    and the last two seconds of every odd clip silent."""
+    n = 480000
+    t = np.arange(n, dtype=np.float64) / 16000.0
+    out = np.empty((batch, n), np.float32)
+    for b in range(batch):
+        noise = normal_f32(seed, 3 * b, n, std=0.05).astype(np.float64)
+        env = np.repeat(uniform_f32(seed, 3 * b + 1, 60).astype(np.float64), n // 60)
+        u = uniform_f32(seed, 3 * b + 2, 2).astype(np.float64)
+        tone = (0.05 + 0.3 * u[1]) * np.sin(2.0 * np.pi * (100.0 + 7000.0 * u[0]) * t)
+        x = (noise * env + tone).astype(np.float32)
+        if b % 2:
+            x[-32000:] = 0.0
+        out[b] = x
+    return out
