@@ -126,7 +126,7 @@ enc_status validate_config(const enc_config* c) {
   if (c->n_mels <= 0 || c->d_model <= 0 || c->n_layers < 0 || c->n_heads <= 0 || c->ffn_dim <= 0 ||
       c->max_frames <= 0 || c->max_batch <= 0)
     return ENC_ERR_INVALID_ARG;
-  if (c->pool_step != 1 && c->pool_step != 2) return ENC_ERR_UNSUPPORTED;
+  if (c->pool_step != 1 && c->pool_step != 2 && c->pool_step != 4) return ENC_ERR_UNSUPPORTED;
   if (c->head_dim != 64 || c->n_heads * c->head_dim != c->d_model) return ENC_ERR_UNSUPPORTED;
   if (c->d_model % 128 || c->d_model > 2048) return ENC_ERR_UNSUPPORTED;
   if (c->ffn_dim % 128) return ENC_ERR_UNSUPPORTED;

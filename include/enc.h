@@ -81,7 +81,7 @@ typedef struct enc_config {
   int32_t ffn_dim;       /* encoder_ffn_dim, multiple of 128 */
   int32_t max_frames;    /* T: mel frames of every clip, zero padded (3000 for 30 s) */
   int32_t max_batch;     /* largest B that enc_forward will be given */
-  int32_t pool_step;     /* 1 (none) or 2 (audio_pool_step) */
+  int32_t pool_step;     /* 1 (none), 2 (audio_pool_step: 25 Hz) or 4 (12.5 Hz) */
   int32_t proj_hidden;   /* 0 = no projector, else hidden width (multiple of 128) */
   int32_t proj_out;      /* projector output width (multiple of 128) */
   float ln_eps;          /* LayerNorm epsilon (1e-5) */
@@ -134,10 +134,11 @@ ENC_API enc_status enc_create(const enc_config *cfg, const enc_weights *w, enc_h
  *            Read during the call; the caller may reuse it on return.
  *   B        1 <= B <= cfg.max_batch
  *   out      device [B, P_out, d_out], cfg.dtype, where
- *              P = ceil(T/2), P_out = P (pool_step 1) or floor(P/2) (pool_step 2),
+ *              P = ceil(T/2), P_out = floor(P / pool_step),
  *              d_out = proj_out if a projector is configured, else d_model.
- *            Clip b carries n_b = ceil(lengths[b]/2) positions (floor(n_b/2)
- *            after pooling); its rows past that count are written as exact zeros.
+ *            Clip b carries n_b = ceil(lengths[b]/2) positions
+ *            (floor(n_b / pool_step) after pooling: only complete windows of
+ *            valid positions); its rows past that count are written as exact zeros.
  * mel and out must stay valid until the stream work has completed. One forward
  * may be in flight per handle at a time (the workspace is shared); handles are
  * independent of each other. Host-detectable errors return before enqueueing.

@@ -147,8 +147,8 @@ class EncoderConfig:
         return dataclasses.replace(self, **kw)
 
 
-# Five workloads: tiny fp32 check case, MiniCPM-o medium tower with pool,
-# Whisper-large tower, Whisper-large + Voxtral projector, ragged sweep.
+# Workloads: tiny fp32 check case, MiniCPM-o medium tower with pool, Whisper-large
+# tower, Whisper-large + Voxtral projector, ragged sweep, Whisper-large at 12.5 Hz.
 CONFIGS = {
     "tiny_fp32": EncoderConfig("tiny_fp32", 128, 1280, 2, 20, 5120, 200, 1, "fp32", 0),
     "medium_pool": EncoderConfig("medium_pool", 80, 1024, 24, 16, 4096, 3000, 8, "bf16", 1,
@@ -158,8 +158,11 @@ CONFIGS = {
                                     proj_hidden=3072, proj_out=3072),
     "large_ragged_b64": EncoderConfig("large_ragged_b64", 128, 1280, 32, 20, 5120, 3000, 64, "bf16", 4,
                                       ragged=(500, 3000)),
+    # rate reduction to 12.5 Hz (Kimi-Audio-7B-Instruct: "Whisper encoder (downsampled to 12.5Hz)")
+    "large_pool4_b16": EncoderConfig("large_pool4_b16", 128, 1280, 32, 20, 5120, 3000, 16, "bf16", 6,
+                                     pool_step=4),
 }
-CONFIG_ORDER = ["tiny_fp32", "medium_pool", "large_b16", "large_proj_b32", "large_ragged_b64"]
+CONFIG_ORDER = ["tiny_fp32", "medium_pool", "large_b16", "large_proj_b32", "large_ragged_b64", "large_pool4_b16"]
 
 LAYER_TENSORS = ["ln1_g", "ln1_b", "q_w", "q_b", "k_w", "v_w", "v_b", "o_w", "o_b",
                  "ln2_g", "ln2_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b"]

@@ -27,6 +27,8 @@ SMALL = [
     (_small("small_pool", pool_step=2, frames=301), [301, 300, 7]),
     (_small("small_proj", proj_hidden=384, proj_out=256), [333, 129, 2]),
     (_small("small_pool_proj", pool_step=2, proj_hidden=256, proj_out=384, d_model=384, n_heads=6), [333, 50, 3]),
+    (_small("small_pool4", pool_step=4, frames=333), [333, 302, 9]),
+    (_small("small_pool4_fp32", pool_step=4, frames=250, dtype="fp32"), [250, 247, 8]),
     (_small("small_fp32", dtype="fp32"), [333, 200, 1]),
     (_small("small_fp32_pool_proj", dtype="fp32", pool_step=2, proj_hidden=256, proj_out=128), [333, 31, 4]),
     (_small("peaky_fp32", weight_std=0.2, frames=260, dtype="fp32"), [260, 131, 65]),
@@ -121,7 +123,8 @@ def test_argument_errors():
 
 
 # ------------------------------------------------------------- full sizes
-FULL = [("medium_pool", [0]), ("large_b16", [5]), ("large_proj_b32", [31]), ("large_ragged_b64", None)]
+FULL = [("medium_pool", [0]), ("large_b16", [5]), ("large_proj_b32", [31]), ("large_ragged_b64", None),
+        ("large_pool4_b16", [3])]
 
 
 @pytest.mark.parametrize("name,sample", FULL, ids=[n for n, _ in FULL])

@@ -296,7 +296,8 @@ def _torch_tower(w, mel, length, d, heads, layers, pool, proj):
 
 
 @pytest.mark.parametrize("t,length,pool,proj", [(37, 37, 1, None), (37, 23, 1, None), (40, 40, 2, None),
-                                                (41, 30, 2, None), (36, 36, 1, (48, 40)), (29, 17, 2, (48, 40))])
+                                                (41, 30, 2, None), (36, 36, 1, (48, 40)), (29, 17, 2, (48, 40)),
+                                                (48, 48, 4, None), (45, 29, 4, None), (43, 40, 4, (48, 40))])
 def test_tower_matches_torch_layers(t, length, pool, proj):
     d, m, f, heads, layers = 128, 8, 256, 2, 2
     w = _rand_weights(d, m, f, layers, proj)
