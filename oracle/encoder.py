@@ -161,14 +161,30 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, n_heads: int, n_valid
     return out
 
 
+def chunked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, n_heads: int, chunk: int,
+                      head_dim: int = 64) -> np.ndarray:
+    """Block-local attention of one clip (MiniCPM-o-2.6, "(2) AUDIO": audio_chunk_length
+    1.0 s): position i attends only to the positions of its own chunk
+    [chunk * floor(i / chunk), chunk * floor(i / chunk) + chunk), a block-diagonal mask."""
+    s = q.shape[0]
+    out = np.zeros((s, n_heads * head_dim), np.float64)
+    for c0 in range(0, s, chunk):
+        c1 = min(s, c0 + chunk)
+        out[c0:c1] = attention(q[c0:c1], k[c0:c1], v[c0:c1], n_heads, None, head_dim)
+    return out
+
+
 # ------------------------------------------------------------------ blocks
-def encoder_layer(x: np.ndarray, lw: dict, n_heads: int, eps: float, head_dim: int = 64) -> np.ndarray:
-    """One pre-LN block on the valid rows x [n, d] of a clip."""
+def encoder_layer(x: np.ndarray, lw: dict, n_heads: int, eps: float, head_dim: int = 64,
+                  attn_chunk: int = 0) -> np.ndarray:
+    """One pre-LN block on the valid rows x [n, d] of a clip (attn_chunk > 0: block-local attention)."""
     a = layer_norm(x, lw["ln1_g"], lw["ln1_b"], eps)
     q = linear(a, lw["q_w"], lw["q_b"])
     k = linear(a, lw["k_w"], None)
     v = linear(a, lw["v_w"], lw["v_b"])
-    x = x + linear(attention(q, k, v, n_heads, None, head_dim), lw["o_w"], lw["o_b"])
+    att = (chunked_attention(q, k, v, n_heads, attn_chunk, head_dim) if attn_chunk > 0
+           else attention(q, k, v, n_heads, None, head_dim))
+    x = x + linear(att, lw["o_w"], lw["o_b"])
     a = layer_norm(x, lw["ln2_g"], lw["ln2_b"], eps)
     return x + linear(gelu(linear(a, lw["fc1_w"], lw["fc1_b"])), lw["fc2_w"], lw["fc2_b"])
 
@@ -187,14 +203,16 @@ def avg_pool(x: np.ndarray, step: int) -> np.ndarray:
 def encode_clip(cfg, w: dict, mel: np.ndarray, length: int, layers: int | None = None) -> np.ndarray:
     """Encoder output of one clip, [P_out, d_out]; rows past the valid count are 0.
 
-    cfg carries the geometry (n_heads, n_layers, frames, pool_step, proj_*, ln_eps).
+    cfg carries the geometry (n_heads, n_layers, frames, pool_step, proj_*, ln_eps,
+    and attn_chunk: 0 for full attention, else the block-local chunk in positions).
     `layers` (default all) limits the number of blocks, for timing samples.
     """
     p = encoder_positions(mel.shape[1])
     n = valid_positions(length)
+    chunk = getattr(cfg, "attn_chunk", 0)
     x = conv_stem(mel, length, w)[:n]                     # key-padding mask: keep valid rows
     for l in range(cfg.n_layers if layers is None else layers):
-        x = encoder_layer(x, layer_weights(w, l), cfg.n_heads, cfg.ln_eps, cfg.head_dim)
+        x = encoder_layer(x, layer_weights(w, l), cfg.n_heads, cfg.ln_eps, cfg.head_dim, chunk)
     y = layer_norm(x, w["lnpost_g"], w["lnpost_b"], cfg.ln_eps)
     p_out = pooled_positions(p, cfg.pool_step)
     if cfg.pool_step > 1:

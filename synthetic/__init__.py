@@ -138,6 +138,7 @@ class EncoderConfig:
     head_dim: int = 64
     ln_eps: float = 1e-5
     weight_std: float = 0.02
+    attn_chunk: int = 0           # 0: full attention; else block-local chunks of this many positions
 
     @property
     def positions(self) -> int:       # conv2 (k3, s2, p1) output length
@@ -148,7 +149,8 @@ class EncoderConfig:
 
 
 # Workloads: tiny fp32 check case, MiniCPM-o medium tower with pool, Whisper-large
-# tower, Whisper-large + Voxtral projector, ragged sweep, Whisper-large at 12.5 Hz.
+# tower, Whisper-large + Voxtral projector, ragged sweep, Whisper-large at 12.5 Hz,
+# MiniCPM-o medium tower with 1 s block-local attention.
 CONFIGS = {
     "tiny_fp32": EncoderConfig("tiny_fp32", 128, 1280, 2, 20, 5120, 200, 1, "fp32", 0),
     "medium_pool": EncoderConfig("medium_pool", 80, 1024, 24, 16, 4096, 3000, 8, "bf16", 1,
@@ -161,8 +163,13 @@ CONFIGS = {
     # rate reduction to 12.5 Hz (Kimi-Audio-7B-Instruct: "Whisper encoder (downsampled to 12.5Hz)")
     "large_pool4_b16": EncoderConfig("large_pool4_b16", 128, 1280, 32, 20, 5120, 3000, 16, "bf16", 6,
                                      pool_step=4),
+    # MiniCPM-o tower with block-local attention over 1 s chunks (50 positions):
+    # MiniCPM-o-2.6, "(2) AUDIO", audio_chunk_length 1.0
+    "medium_chunk50": EncoderConfig("medium_chunk50", 80, 1024, 24, 16, 4096, 3000, 8, "bf16", 7,
+                                    pool_step=2, attn_chunk=50),
 }
-CONFIG_ORDER = ["tiny_fp32", "medium_pool", "large_b16", "large_proj_b32", "large_ragged_b64", "large_pool4_b16"]
+CONFIG_ORDER = ["tiny_fp32", "medium_pool", "large_b16", "large_proj_b32", "large_ragged_b64", "large_pool4_b16",
+                "medium_chunk50"]
 
 LAYER_TENSORS = ["ln1_g", "ln1_b", "q_w", "q_b", "k_w", "v_w", "v_b", "o_w", "o_b",
                  "ln2_g", "ln2_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b"]

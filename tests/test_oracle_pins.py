@@ -23,9 +23,11 @@ RNG = np.random.default_rng(1234)
 class Geo:
     """Minimal geometry object accepted by oracle.encode_clip."""
 
-    def __init__(self, n_layers, n_heads, pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64):
+    def __init__(self, n_layers, n_heads, pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64,
+                 attn_chunk=0):
         self.n_layers, self.n_heads, self.pool_step = n_layers, n_heads, pool_step
         self.proj_hidden, self.proj_out, self.ln_eps, self.head_dim = proj_hidden, proj_out, ln_eps, head_dim
+        self.attn_chunk = attn_chunk
 
 
 # ------------------------------------------------------------------ counts
@@ -252,8 +254,9 @@ def _rand_weights(d, m, f, layers, proj=None, std=0.2):
     return w
 
 
-def _torch_tower(w, mel, length, d, heads, layers, pool, proj):
-    """Independent composition from torch.nn layers (float64)."""
+def _torch_tower(w, mel, length, d, heads, layers, pool, proj, chunk=0):
+    """Independent composition from torch.nn layers (float64); chunk > 0 adds a
+    block-diagonal attention mask (positions attend within their own chunk)."""
     T = lambda a: torch.tensor(np.asarray(a, np.float64))
     m, t = mel.shape
     c1 = torch.nn.Conv1d(m, d, 3, padding=1); c2 = torch.nn.Conv1d(d, d, 3, stride=2, padding=1)
@@ -281,10 +284,17 @@ def _torch_tower(w, mel, length, d, heads, layers, pool, proj):
         lay.eval()
         enc.append(lay)
     pad = torch.zeros(1, p, dtype=torch.bool); pad[0, n:] = True
+    blocks = None
     y = h[None]
+    if chunk:
+        # the valid rows alone (a padded query whose chunk holds no valid key would
+        # give NaN, and NaN values reach valid rows through zero probabilities)
+        y, pad = h[None, :n], None
+        idx = torch.arange(n) // chunk
+        blocks = idx[:, None] != idx[None, :]           # True: not allowed to attend
     with torch.no_grad():
         for lay in enc:
-            y = lay(y, src_key_padding_mask=pad)
+            y = lay(y, src_mask=blocks, src_key_padding_mask=pad)
         y = torch.nn.functional.layer_norm(y, (d,), T(w["lnpost_g"]), T(w["lnpost_b"]), 1e-5)[0]
         y = y[:n]
         if pool > 1:
@@ -295,16 +305,18 @@ def _torch_tower(w, mel, length, d, heads, layers, pool, proj):
     return y.numpy()
 
 
-@pytest.mark.parametrize("t,length,pool,proj", [(37, 37, 1, None), (37, 23, 1, None), (40, 40, 2, None),
-                                                (41, 30, 2, None), (36, 36, 1, (48, 40)), (29, 17, 2, (48, 40)),
-                                                (48, 48, 4, None), (45, 29, 4, None), (43, 40, 4, (48, 40))])
-def test_tower_matches_torch_layers(t, length, pool, proj):
+@pytest.mark.parametrize("t,length,pool,proj,chunk", [
+    (37, 37, 1, None, 0), (37, 23, 1, None, 0), (40, 40, 2, None, 0), (41, 30, 2, None, 0),
+    (36, 36, 1, (48, 40), 0), (29, 17, 2, (48, 40), 0), (48, 48, 4, None, 0), (45, 29, 4, None, 0),
+    (43, 40, 4, (48, 40), 0),
+    (49, 49, 1, None, 7), (47, 33, 2, None, 5), (40, 31, 1, (48, 40), 6)])   # block-local attention
+def test_tower_matches_torch_layers(t, length, pool, proj, chunk):
     d, m, f, heads, layers = 128, 8, 256, 2, 2
     w = _rand_weights(d, m, f, layers, proj)
     mel = RNG.uniform(-1.5, 1.5, (m, t))
-    geo = Geo(layers, heads, pool, *(proj or (0, 0)))
+    geo = Geo(layers, heads, pool, *(proj or (0, 0)), attn_chunk=chunk)
     got = O.encode_clip(geo, w, mel, length)
-    ref = _torch_tower(w, mel, length, d, heads, layers, pool, proj)
+    ref = _torch_tower(w, mel, length, d, heads, layers, pool, proj, chunk)
     nv = O.valid_output_rows(geo, length)
     assert got.shape[0] == O.pooled_positions(O.encoder_positions(t), pool)
     assert nv == ref.shape[0]
@@ -332,3 +344,20 @@ def test_layer_limit_and_zero_layers():
     y0 = O.encode_clip(geo, w, mel, 20, layers=0)
     stem = O.conv_stem(mel, 20, w)
     np.testing.assert_allclose(y0, O.layer_norm(stem, w["lnpost_g"], w["lnpost_b"]), atol=1e-14)
+
+
+def test_chunked_attention_special_cases():
+    """Block-local attention: a chunk covering the clip is full attention; a chunk of
+    one position returns v itself (softmax over one key is 1); keys outside a
+    chunk change nothing inside it."""
+    s_len, heads = 23, 2
+    q, k, v = (RNG.standard_normal((s_len, 64 * heads)) for _ in range(3))
+    np.testing.assert_array_equal(O.chunked_attention(q, k, v, heads, 23), O.attention(q, k, v, heads))
+    np.testing.assert_array_equal(O.chunked_attention(q, k, v, heads, 100), O.attention(q, k, v, heads))
+    np.testing.assert_allclose(O.chunked_attention(q, k, v, heads, 1), v, rtol=0, atol=1e-15)
+    k2, v2 = k.copy(), v.copy()
+    k2[10:], v2[10:] = 7.0, -3.0                        # chunks of 5: rows 0..9 are chunks 0 and 1
+    a = O.chunked_attention(q, k, v, heads, 5)
+    b = O.chunked_attention(q, k2, v2, heads, 5)
+    np.testing.assert_array_equal(a[:10], b[:10])
+    assert not np.allclose(a[10:], b[10:])
