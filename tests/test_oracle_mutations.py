@@ -67,7 +67,7 @@ def _conv_shifted(x, w, b, stride):
     return np.roll(y, 1, axis=1)
 
 
-def _post_ln_layer(x, lw, n_heads, eps, head_dim=64):
+def _post_ln_layer(x, lw, n_heads, eps, head_dim=64, attn_chunk=0):
     q = E.linear(x, lw["q_w"], lw["q_b"]); k = E.linear(x, lw["k_w"], None); v = E.linear(x, lw["v_w"], lw["v_b"])
     x = E.layer_norm(x + E.linear(E.attention(q, k, v, n_heads, None, head_dim), lw["o_w"], lw["o_b"]),
                      lw["ln1_g"], lw["ln1_b"], eps)
@@ -75,7 +75,7 @@ def _post_ln_layer(x, lw, n_heads, eps, head_dim=64):
                         lw["ln2_g"], lw["ln2_b"], eps)
 
 
-def _k_biased_layer(x, lw, n_heads, eps, head_dim=64):
+def _k_biased_layer(x, lw, n_heads, eps, head_dim=64, attn_chunk=0):
     lw = dict(lw); lw["k_b"] = lw["q_b"]
     a = E.layer_norm(x, lw["ln1_g"], lw["ln1_b"], eps)
     q = E.linear(a, lw["q_w"], lw["q_b"]); k = E.linear(a, lw["k_w"], lw["k_b"]); v = E.linear(a, lw["v_w"], lw["v_b"])
