@@ -39,7 +39,7 @@ class EncConfig(ctypes.Structure):
                 ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ffn_dim", ctypes.c_int32),
                 ("max_frames", ctypes.c_int32), ("max_batch", ctypes.c_int32), ("pool_step", ctypes.c_int32),
                 ("proj_hidden", ctypes.c_int32), ("proj_out", ctypes.c_int32), ("ln_eps", ctypes.c_float),
-                ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32), ("attn_chunk", ctypes.c_int32)]
 
 
 _VP = ctypes.c_void_p
@@ -138,11 +138,11 @@ class Encoder:
     """
 
     def __init__(self, *, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
-                 pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, weights: dict):
+                 pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0, weights: dict):
         self.lib = load_library()
         self.cfg = EncConfig(n_mels, d_model, n_layers, n_heads, head_dim, ffn_dim, max_frames, max_batch,
                              pool_step, proj_hidden, proj_out, ln_eps,
-                             ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0)
+                             ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0, attn_chunk)
         w = EncWeights()
         for f in ("conv1_w", "conv1_b", "conv2_w", "conv2_b", "lnpost_g", "lnpost_b",
                   "proj1_w", "proj1_b", "proj2_w", "proj2_b"):

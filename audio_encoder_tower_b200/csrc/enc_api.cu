@@ -48,7 +48,8 @@ struct enc_handle {
   void* y1 = nullptr;        // [max_batch * Tp + 2, d]
   float* x = nullptr;        // [max_batch * P, d] residual stream
   void *a = nullptr, *qkv = nullptr, *o = nullptr, *f = nullptr, *e = nullptr, *p1 = nullptr;
-  int* meta = nullptr;       // device [cu (B+1) | cu_out (B+1) | len (B)]
+  int* meta = nullptr;       // device [cu (B+1) | cu_out (B+1) | len (B) | cu_attn (segments+1)]
+  int meta_ints = 0;         // capacity of meta / h_meta
   int* h_meta = nullptr;     // pinned host staging of meta
   int* status = nullptr;     // device status word
   cudaEvent_t meta_free = nullptr;
@@ -134,6 +135,12 @@ enc_status validate_config(const enc_config* c) {
   if (c->proj_hidden < 0 || c->proj_out < 0) return ENC_ERR_INVALID_ARG;
   if (c->proj_hidden && (c->proj_hidden % 128 || c->proj_out <= 0 || c->proj_out % 128)) return ENC_ERR_UNSUPPORTED;
   if (!(c->ln_eps > 0.f)) return ENC_ERR_INVALID_ARG;
+  // block-local attention: every chunk is one attention segment (grid z <= 65535)
+  if (c->attn_chunk < 0) return ENC_ERR_INVALID_ARG;
+  if (c->attn_chunk > 0) {
+    const long long p = (c->max_frames + 1) / 2;
+    if ((long long)c->max_batch * ((p + c->attn_chunk - 1) / c->attn_chunk) > 65535) return ENC_ERR_UNSUPPORTED;
+  }
   // index arithmetic stays in 32 bits
   const long long rows = (long long)c->max_batch * (c->max_frames + 4);
   if (rows * (long long)(3 * c->d_model > c->ffn_dim ? 3 * c->d_model : c->ffn_dim) > (1ll << 31) - 1)
@@ -234,10 +241,12 @@ enc_status build(enc_handle* h, const enc_weights* w) {
   ENC_TRY(cudaMemset(h->qkv, 0, (size_t)rows_p * 3 * d * h->esz));
   ENC_TRY(cudaMemset(h->o, 0, (size_t)rows_p * d * h->esz));
   ENC_TRY(cudaMemset(h->f, 0, (size_t)rows_p * F * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->meta, (size_t)(3 * Bm + 2) * 4));
+  // block-local attention adds the chunk boundaries: at most ceil(P / chunk) per clip
+  h->meta_ints = 3 * Bm + 2 + (c.attn_chunk > 0 ? Bm * ((h->P + c.attn_chunk - 1) / c.attn_chunk) + 1 : 0);
+  ENC_CHECK(dev_alloc(h, &h->meta, (size_t)h->meta_ints * 4));
   ENC_CHECK(dev_alloc(h, &h->status, 4));
   ENC_TRY(cudaMemset(h->status, 0, 4));
-  if (cudaMallocHost(&h->h_meta, (size_t)(3 * Bm + 2) * 4) != cudaSuccess) {
+  if (cudaMallocHost(&h->h_meta, (size_t)h->meta_ints * 4) != cudaSuccess) {
     cudaGetLastError();
     h->h_meta = nullptr;
     return ENC_ERR_OOM;
@@ -322,7 +331,55 @@ cudaError_t run(enc_handle* h, cudaStream_t s, int cls, double flops, F&& launch
 struct Work {
   int B, R, R_out, max_n;
   double sum_n2;
+  int nseg, max_seg;   // attention segments: the clips, or their chunks with block-local attention
+  double sum_seg2;
 };
+
+int valid_out(const enc_handle* h, int n);   // output rows of a clip with n positions
+
+// Per-clip counts of one batch, staged into hm for upload:
+//   [cu (B+1) | cu_out (B+1) | len (B) | cu_attn (nseg+1), block-local attention only]
+// n_b = ceil(len_b / 2) positions; cu_attn cuts every clip into chunks of
+// cfg.attn_chunk positions (the last one shorter). Returns the ints to upload,
+// or 0 when a length is outside [1, T].
+int stage_meta(const enc_handle* h, const int32_t* lengths, int B, int* hm, Work* wk) {
+  int* cu = hm;
+  int* cu_out = hm + (B + 1);
+  int* len = hm + 2 * (B + 1);
+  int max_n = 0;
+  double sum_n2 = 0.0;
+  cu[0] = cu_out[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    len[b] = lengths ? lengths[b] : h->T;
+    if (len[b] < 1 || len[b] > h->T) return 0;
+    const int n = (len[b] + 1) / 2;
+    cu[b + 1] = cu[b] + n;
+    cu_out[b + 1] = cu_out[b] + valid_out(h, n);
+    if (n > max_n) max_n = n;
+    sum_n2 += (double)n * n;
+  }
+  int total = 3 * B + 2;
+  int nseg = B, max_seg = max_n;
+  double sum_seg2 = sum_n2;
+  const int chunk = h->cfg.attn_chunk;
+  if (chunk > 0) {
+    int* ca = hm + total;
+    nseg = 0;
+    max_seg = 0;
+    sum_seg2 = 0.0;
+    ca[0] = 0;
+    for (int b = 0; b < B; ++b)
+      for (int c0 = cu[b]; c0 < cu[b + 1]; c0 += chunk) {
+        const int c1 = c0 + chunk < cu[b + 1] ? c0 + chunk : cu[b + 1];
+        ca[++nseg] = c1;
+        if (c1 - c0 > max_seg) max_seg = c1 - c0;
+        sum_seg2 += (double)(c1 - c0) * (c1 - c0);
+      }
+    total += nseg + 1;
+  }
+  *wk = Work{B, cu[B], cu_out[B], max_n, sum_n2, nseg, max_seg, sum_seg2};
+  return total;
+}
 
 enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& wk, cudaStream_t s) {
   const enc_config& c = h->cfg;
@@ -331,6 +388,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
   const int* cu = h->meta;
   const int* cu_out = h->meta + (B + 1);
   const int* len = h->meta + 2 * (B + 1);
+  const int* cu_att = c.attn_chunk > 0 ? h->meta + 3 * B + 2 : cu;   // attention segments
   bf16* melT_data = reinterpret_cast<bf16*>(h->melT) + M;
   ENC_RUN(ENC_K_MEL, 0.0,
           launch_mel_stage<bf16>(reinterpret_cast<const bf16*>(mel), len, melT_data, B, M, h->T, h->Tp, s));
@@ -359,8 +417,9 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
     g.epi = epi_base(EPI_STORE);
     g.epi.bias = h->qkv_b[l]; g.epi.out = h->qkv; g.epi.ldo = 3 * d;
     ENC_RUN(ENC_K_QKV, 6.0 * Rd * d, launch_gemm_tc(h->m_a, lm.qkv, g, h->sm_count, s, &h->m_out_qkv));
-    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d,
-            launch_attention_tc(h->m_qkv, reinterpret_cast<bf16*>(h->o), cu, B, wk.max_n, d, c.n_heads, h->status, s));
+    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_seg2 * d,
+            launch_attention_tc(h->m_qkv, reinterpret_cast<bf16*>(h->o), cu_att, wk.nseg, wk.max_seg, d, c.n_heads,
+                                h->status, s));
     g.N = d; g.num_kb = d / 64;
     g.epi = epi_base(EPI_RESIDUAL);
     g.epi.bias = h->o_b[l]; g.epi.resid = h->x; g.epi.ldo = d;
@@ -408,6 +467,7 @@ enc_status forward_f32(enc_handle* h, const void* mel, void* out, const Work& wk
   const int* cu = h->meta;
   const int* cu_out = h->meta + (B + 1);
   const int* len = h->meta + 2 * (B + 1);
+  const int* cu_att = c.attn_chunk > 0 ? h->meta + 3 * B + 2 : cu;   // attention segments
   float* melT = reinterpret_cast<float*>(h->melT);
   float* y1 = reinterpret_cast<float*>(h->y1);
   ENC_RUN(ENC_K_MEL, 0.0,
@@ -434,7 +494,8 @@ enc_status forward_f32(enc_handle* h, const void* mel, void* out, const Work& wk
     e.bias = h->qkv_b[l]; e.out = qkv; e.ldo = 3 * d;
     ENC_RUN(ENC_K_QKV, 6.0 * Rd * d,
             launch_sgemm(a, d, reinterpret_cast<const float*>(h->qkv_w[l]), d, R, 3 * d, d, e, s));
-    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_n2 * d, launch_attention_f32(qkv, o, cu, B, wk.max_n, d, c.n_heads, s));
+    ENC_RUN(ENC_K_ATTN, 4.0 * wk.sum_seg2 * d,
+            launch_attention_f32(qkv, o, cu_att, wk.nseg, wk.max_seg, d, c.n_heads, s));
     e = epi_base(EPI_RESIDUAL);
     e.bias = h->o_b[l]; e.resid = h->x; e.ldo = d;
     ENC_RUN(ENC_K_OUT, 2.0 * Rd * d, launch_sgemm(o, d, reinterpret_cast<const float*>(h->o_w[l]), d, R, d, d, e, s));
@@ -546,31 +607,15 @@ enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, i
                        cudaStream_t stream) {
   if (!h || !mel || !out || B < 1 || B > h->cfg.max_batch) return ENC_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(mel) | reinterpret_cast<uintptr_t>(out)) & 15u) return ENC_ERR_INVALID_ARG;
-  // per-clip counts (host): n_b = ceil(len_b / 2) positions, packed offsets
-  std::vector<int> len(B), cu(B + 1), cu_out(B + 1);
-  int max_n = 0;
-  double sum_n2 = 0.0;
-  cu[0] = cu_out[0] = 0;
-  for (int b = 0; b < B; ++b) {
-    len[b] = lengths ? lengths[b] : h->T;
-    if (len[b] < 1 || len[b] > h->T) return ENC_ERR_INVALID_ARG;
-    const int n = (len[b] + 1) / 2;
-    cu[b + 1] = cu[b] + n;
-    cu_out[b + 1] = cu_out[b] + valid_out(h, n);
-    if (n > max_n) max_n = n;
-    sum_n2 += (double)n * n;
-  }
   if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
   // the pinned staging buffer may still feed the previous forward's upload
   if (h->meta_pending) ENC_TRY(cudaEventSynchronize(h->meta_free));
-  int* hm = h->h_meta;
-  memcpy(hm, cu.data(), (B + 1) * 4);
-  memcpy(hm + B + 1, cu_out.data(), (B + 1) * 4);
-  memcpy(hm + 2 * (B + 1), len.data(), B * 4);
-  ENC_TRY(cudaMemcpyAsync(h->meta, hm, (size_t)(3 * B + 2) * 4, cudaMemcpyHostToDevice, stream));
+  Work wk;
+  const int nints = stage_meta(h, lengths, B, h->h_meta, &wk);
+  if (nints == 0) return ENC_ERR_INVALID_ARG;
+  ENC_TRY(cudaMemcpyAsync(h->meta, h->h_meta, (size_t)nints * 4, cudaMemcpyHostToDevice, stream));
   ENC_TRY(cudaEventRecord(h->meta_free, stream));
   h->meta_pending = true;
-  const Work wk{B, cu[B], cu_out[B], max_n, sum_n2};
   return h->bf16 ? forward_bf16(h, mel, out, wk, stream) : forward_f32(h, mel, out, wk, stream);
 }
 
@@ -683,21 +728,10 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
 
   // per-clip counts, written straight into the handle's pinned staging buffer
   if (h->meta_pending) ENC_TRY(cudaEventSynchronize(h->meta_free));
-  int* hcu = h->h_meta;
-  int* hcu_out = hcu + (B + 1);
-  int* hlen = hcu + 2 * (B + 1);
-  int max_n = 0;
-  double sum_n2 = 0.0;
-  hcu[0] = hcu_out[0] = 0;
-  for (int b = 0; b < B; ++b) {
-    hlen[b] = lengths ? lengths[b] : h->T;
-    const int n = (hlen[b] + 1) / 2;
-    hcu[b + 1] = hcu[b] + n;
-    hcu_out[b + 1] = hcu_out[b] + valid_out(h, n);
-    if (n > max_n) max_n = n;
-    sum_n2 += (double)n * n;
-  }
-  const int R = hcu[B], R_out = hcu_out[B];
+  Work wk;
+  const int nints = stage_meta(h, lengths, B, h->h_meta, &wk);
+  if (nints == 0) return ENC_ERR_INVALID_ARG;
+  const int R = wk.R, R_out = wk.R_out;
 
   // carve the workspace of this batch out of the static array
   const size_t rows_t = (size_t)B * h->Tp;
@@ -712,7 +746,7 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   unsigned char* f = take((size_t)R * F * h->esz);
   unsigned char* e = c.proj_hidden ? take((size_t)R_out * d * h->esz) : nullptr;
   unsigned char* p1 = c.proj_hidden ? take((size_t)R_out * c.proj_hidden * h->esz) : nullptr;
-  unsigned char* meta = take((size_t)(3 * B + 2) * 4);
+  unsigned char* meta = take((size_t)nints * 4);
   if (off > ENC_STATIC_SCRATCH_BYTES) return ENC_ERR_INVALID_ARG;   // batch too large for the array
 
   // the array keeps the previous call's contents: clear what is read as zero
@@ -753,13 +787,12 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
     if (!ok) st = ENC_ERR_CUDA;
   }
   if (st == ENC_OK) {
-    cudaError_t ce = cudaMemcpyAsync(h->meta, h->h_meta, (size_t)(3 * B + 2) * 4, cudaMemcpyHostToDevice, stream);
+    cudaError_t ce = cudaMemcpyAsync(h->meta, h->h_meta, (size_t)nints * 4, cudaMemcpyHostToDevice, stream);
     if (ce == cudaSuccess) ce = cudaEventRecord(h->meta_free, stream);
     if (ce != cudaSuccess) st = cuda_status(ce);
     else h->meta_pending = true;
   }
   if (st == ENC_OK) {
-    const Work wk{B, R, R_out, max_n, sum_n2};
     st = h->bf16 ? forward_bf16(h, mel, out, wk, stream) : forward_f32(h, mel, out, wk, stream);
   }
   h->melT = s_melT; h->y1 = s_y1; h->x = s_x; h->a = s_a; h->qkv = s_qkv; h->o = s_o; h->f = s_f; h->e = s_e;

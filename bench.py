@@ -48,7 +48,9 @@ def workload_flops(cfg, lengths, layers=None) -> float:
     for ln in lengths:
         n = (int(ln) + 1) // 2
         total += 2.0 * (2 * n) * d * 3 * m + 2.0 * n * d * 3 * d
-        total += L * (6.0 * n * d * d + 4.0 * n * n * d + 2.0 * n * d * d + 4.0 * n * d * f)
+        c = cfg.attn_chunk if cfg.attn_chunk else n      # block-local attention: per chunk
+        attn = sum(min(c, n - c0) ** 2 for c0 in range(0, n, c))
+        total += L * (6.0 * n * d * d + 4.0 * attn * d + 2.0 * n * d * d + 4.0 * n * d * f)
         if cfg.proj_hidden:
             no = n // cfg.pool_step if cfg.pool_step > 1 else n
             total += 2.0 * no * (d * cfg.proj_hidden + cfg.proj_hidden * cfg.proj_out)
@@ -61,7 +63,8 @@ def workload_desc(cfg, n_gpus):
                      f"FFN{cfg.ffn_dim}, {cfg.n_mels} mel x {cfg.frames} frames, B={cfg.batch} per GPU"
                      + (f", pool {cfg.pool_step}" if cfg.pool_step > 1 else "")
                      + (f", projector {cfg.d_model}->{cfg.proj_hidden}->{cfg.proj_out}" if cfg.proj_hidden else "")
-                     + (f", lengths U[{cfg.ragged[0]},{cfg.ragged[1]}] frames" if cfg.ragged else "")),
+                     + (f", lengths U[{cfg.ragged[0]},{cfg.ragged[1]}] frames" if cfg.ragged else "")
+                     + (f", block-local attention over {cfg.attn_chunk}-position chunks" if cfg.attn_chunk else "")),
         "global_batch": cfg.batch * n_gpus,
         "frames": cfg.frames,
         "positions": cfg.positions,
@@ -318,7 +321,8 @@ def main():
     mel_np = S.make_mel(rcfg)
     enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
                   ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=cfg.batch, dtype=cfg.dtype,
-                  pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out, weights=w_dev)
+                  pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
+                  attn_chunk=cfg.attn_chunk, weights=w_dev)
     del w_dev
     torch.cuda.empty_cache()
     mel = torch.from_numpy(mel_np).to(device=dev, dtype=dt)

@@ -87,6 +87,10 @@ typedef struct enc_config {
   float ln_eps;          /* LayerNorm epsilon (1e-5) */
   int32_t dtype;         /* enc_dtype */
   uint32_t flags;        /* reserved, must be 0 */
+  int32_t attn_chunk;    /* 0: full bidirectional attention within each clip; > 0: block-local
+                            attention, position i of a clip attending only within its chunk of
+                            attn_chunk positions (MiniCPM-o-2.6, "(2) AUDIO": audio_chunk_length
+                            1.0 s = 50 positions); max_batch * ceil(P / attn_chunk) <= 65535 */
 } enc_config;
 
 /*

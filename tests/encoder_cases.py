@@ -30,7 +30,7 @@ def make_encoder(cfg, dev_w, max_batch=None):
     return Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
                    ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=max_batch or cfg.batch, dtype=cfg.dtype,
                    pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
-                   ln_eps=cfg.ln_eps, weights=dev_w)
+                   ln_eps=cfg.ln_eps, attn_chunk=cfg.attn_chunk, weights=dev_w)
 
 
 def run_gpu(enc, cfg, mel_np, lengths):

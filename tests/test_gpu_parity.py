@@ -28,6 +28,9 @@ SMALL = [
     (_small("small_proj", proj_hidden=384, proj_out=256), [333, 129, 2]),
     (_small("small_pool_proj", pool_step=2, proj_hidden=256, proj_out=384, d_model=384, n_heads=6), [333, 50, 3]),
     (_small("small_pool4", pool_step=4, frames=333), [333, 302, 9]),
+    (_small("small_chunk", attn_chunk=50, frames=333), [333, 201, 99]),
+    (_small("small_chunk_fp32", attn_chunk=7, frames=100, dtype="fp32"), [100, 57, 13]),
+    (_small("small_chunk1_fp32", attn_chunk=1, frames=40, dtype="fp32"), [40, 9, 2]),
     (_small("small_pool4_fp32", pool_step=4, frames=250, dtype="fp32"), [250, 247, 8]),
     (_small("small_fp32", dtype="fp32"), [333, 200, 1]),
     (_small("small_fp32_pool_proj", dtype="fp32", pool_step=2, proj_hidden=256, proj_out=128), [333, 31, 4]),
@@ -124,7 +127,7 @@ def test_argument_errors():
 
 # ------------------------------------------------------------- full sizes
 FULL = [("medium_pool", [0]), ("large_b16", [5]), ("large_proj_b32", [31]), ("large_ragged_b64", None),
-        ("large_pool4_b16", [3])]
+        ("large_pool4_b16", [3]), ("medium_chunk50", [2])]
 
 
 @pytest.mark.parametrize("name,sample", FULL, ids=[n for n, _ in FULL])
