@@ -22,7 +22,8 @@ ENC_DTYPE_BF16, ENC_DTYPE_FP32 = 0, 1
 EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status", "enc_destroy",
             "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
             "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch",
-            "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy"]
+            "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy",
+            "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy"]
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -105,6 +106,15 @@ def load_library(path: str = LIB_PATH):
     lib.enc_frontend_log_mel.restype = ctypes.c_int
     lib.enc_frontend_destroy.argtypes = [_VP]
     lib.enc_frontend_destroy.restype = None
+    lib.enc_cache_create.argtypes = [_VP, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p)]
+    lib.enc_cache_create.restype = ctypes.c_int
+    lib.enc_forward_cached.argtypes = [_VP, _VP, i32p, ctypes.POINTER(ctypes.c_uint64), ctypes.c_int32, _VP, i32p,
+                                       _VP]
+    lib.enc_forward_cached.restype = ctypes.c_int
+    lib.enc_cache_size.argtypes = [_VP]
+    lib.enc_cache_size.restype = ctypes.c_int32
+    lib.enc_cache_destroy.argtypes = [_VP]
+    lib.enc_cache_destroy.restype = None
     _LIB = lib
     return lib
 
@@ -299,6 +309,50 @@ class Frontend:
     def close(self):
         if self.h:
             self.lib.enc_frontend_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Cache:
+    """Embeddings cache in front of an Encoder (enc_cache_create / enc_forward_cached):
+    outputs looked up by a 64-bit key per clip that identifies its mel and length."""
+
+    def __init__(self, encoder: "Encoder", capacity: int):
+        self.lib = load_library()
+        self.encoder = encoder
+        h = ctypes.c_void_p()
+        _check(self.lib.enc_cache_create(encoder.handle, int(capacity), ctypes.byref(h)), "enc_cache_create")
+        self.h = h
+
+    def forward(self, mel, keys, lengths=None, out=None, stream=None):
+        """Returns (out, hits): hits[b] = 1 where clip b's output came from the cache."""
+        import torch
+        B = int(mel.shape[0])
+        if out is None:
+            _, p_out, d_out = self.encoder.output_positions(B, lengths)
+            out = torch.empty((B, p_out, d_out), dtype=mel.dtype, device=mel.device)
+        k = np.ascontiguousarray(np.asarray(keys, dtype=np.uint64))
+        if k.shape != (B,):
+            raise ValueError("one key per clip")
+        ln = None if lengths is None else np.ascontiguousarray(np.asarray(lengths, dtype=np.int32))
+        hits = np.zeros(B, dtype=np.int32)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        _check(self.lib.enc_forward_cached(self.h, _ptr(mel), None if ln is None else ln.ctypes.data_as(i32p),
+                                           k.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64)), int(B), _ptr(out),
+                                           hits.ctypes.data_as(i32p), _stream_handle(stream)), "enc_forward_cached")
+        return out, hits
+
+    def size(self) -> int:
+        return int(self.lib.enc_cache_size(self.h))
+
+    def close(self):
+        if self.h:
+            self.lib.enc_cache_destroy(self.h)
             self.h = None
 
     def __del__(self):

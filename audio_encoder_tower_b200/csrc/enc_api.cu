@@ -805,3 +805,16 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   h->profile = s_profile;
   return st;
 }
+
+namespace enc {
+bool handle_geometry(const enc_handle* h, HandleGeometry* g) {
+  if (!h || !g) return false;
+  g->n_mels = h->cfg.n_mels;
+  g->frames = h->T;
+  g->max_batch = h->cfg.max_batch;
+  g->device = h->device;
+  g->mel_bytes = (size_t)h->cfg.n_mels * h->T * h->esz;
+  g->out_bytes = (size_t)h->p_out * h->d_out * h->esz;
+  return true;
+}
+}  // namespace enc

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "../../include/enc.h"
 
 namespace enc {
 
@@ -80,6 +81,16 @@ cudaError_t launch_final_ln(const float* x, const float* g, const float* b, cons
 // Zero rows j >= cu_out[b+1] - cu_out[b] of out [B, p_out, width].
 template <typename OutT>
 cudaError_t launch_zero_tail_rows(OutT* out, const int* cu_out, int B, int p_out, int width, cudaStream_t s);
+
+// -------------------------------------------------- encoder handle geometry
+// Sizes of one clip's input and output blocks for an encoder handle (for the
+// embeddings cache, which sits beside the handle). Returns false for a null handle.
+struct HandleGeometry {
+  int n_mels, frames, max_batch, device;
+  size_t mel_bytes;   // one clip of enc_forward's mel input: n_mels x frames elements
+  size_t out_bytes;   // one clip of its output: P_out x d_out elements
+};
+bool handle_geometry(const enc_handle* h, HandleGeometry* g);
 
 // ------------------------------------------------------------ set-up work
 cudaError_t launch_position_table(float* pe, int P, int d, cudaStream_t s);

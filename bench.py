@@ -7,7 +7,7 @@ batch 16 per GPU, bf16 operands with fp32 accumulation, synthetic seeded inputs
 and random weights of that architecture.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
-    python bench.py --kernel qkv|out|fc1|fc2|attention|frontend [--steps K] [--warmup W]   (one step alone)
+    python bench.py --kernel qkv|out|fc1|fc2|attention|frontend|cache [--steps K] [--warmup W]   (one step alone)
 
 One step = one enc_forward over a batch of 16 clips. Multi-GPU (torchrun, one
 process per GPU) runs independent replicas, each with its own batch of 16
@@ -217,14 +217,38 @@ def gemm_traffic_record():
 def run_kernel(args, cfg):
     """Time one step of the workload alone through the C ABI (for profiling): a
     layer GEMM shape (qkv, out, fc1, fc2) at M = batch x positions, the
-    attention, or the log-mel front end over the batch's 30 s clips."""
+    attention, the log-mel front end over the batch's 30 s clips, or the
+    encoder behind its embeddings cache with half of every step's clips seen
+    in the step before."""
     import torch
     from audio_encoder_tower_b200.binding import attention_bf16, linear_bf16
     torch.cuda.set_device(0)
     n = cfg.frames // 2
     M, d, f, H = cfg.batch * n, cfg.d_model, cfg.ffn_dim, cfg.n_heads
     g = torch.Generator(device="cuda").manual_seed(cfg.seed)
-    if args.kernel == "frontend":
+    if args.kernel == "cache":
+        from audio_encoder_tower_b200 import Cache, Encoder
+        w_np = S.make_weights(cfg)
+        w_dev = {k: torch.from_numpy(v).to(device="cuda", dtype=torch.bfloat16) for k, v in w_np.items()}
+        del w_np
+        enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
+                      ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=cfg.batch, dtype=cfg.dtype,
+                      pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
+                      attn_chunk=cfg.attn_chunk, weights=w_dev)
+        del w_dev
+        mel = torch.from_numpy(S.make_mel(cfg)).to(device="cuda", dtype=torch.bfloat16)
+        cache = Cache(enc, 4 * cfg.batch)
+        half, step_no = cfg.batch // 2, [0]
+
+        def launch():   # keys of step i: half * i .. half * i + B - 1 (the first half seen in step i - 1)
+            i = step_no[0]
+            step_no[0] += 1
+            cache.forward(mel, list(range(half * i, half * i + cfg.batch)))
+
+        flops = workload_flops(cfg, S.make_lengths(cfg)[:half])   # the clips computed per step
+        shape = {"clips": cfg.batch, "hits_per_step": half, "capacity": 4 * cfg.batch,
+                 "audio_s": cfg.batch * cfg.frames / FRAMES_PER_SECOND}
+    elif args.kernel == "frontend":
         from audio_encoder_tower_b200 import Frontend
         fe = Frontend(n_mels=cfg.n_mels, max_batch=cfg.batch)
         audio = torch.from_numpy(S.make_audio(cfg.batch)).cuda()
@@ -263,7 +287,7 @@ def run_kernel(args, cfg):
     ms = e0.elapsed_time(e1) / args.steps
     line = {"kernel": args.kernel, "workload": cfg.name, "shape": shape, "launches": args.steps,
             "ms_per_launch": ms, "tflops": flops / ms / 1e9}
-    if args.kernel == "frontend":
+    if args.kernel in ("frontend", "cache"):
         line["audio_s_per_s"] = shape["audio_s"] / (ms / 1e3)
     print(json.dumps(line), flush=True)
 
@@ -277,7 +301,7 @@ def main():
     ap.add_argument("--config", default="large_b16", choices=S.CONFIG_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention", "frontend"],
+    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention", "frontend", "cache"],
                     help="time one layer kernel of the workload alone (profiling aid)")
     args = ap.parse_args()
     cfg = S.CONFIGS[args.config]

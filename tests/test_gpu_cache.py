@@ -1,0 +1,72 @@
+"""Embeddings cache (include/enc_cache.h) on the GPU: hits return exactly what
+enc_forward computes for the clip (bit for bit: the encoder's result for a clip
+does not depend on its batch), repeated keys are computed once, the least
+recently used entry is replaced when the cache is full."""
+import numpy as np
+import pytest
+
+import synthetic as S
+from tests.encoder_cases import make_encoder, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(capacity):
+    import torch
+    from audio_encoder_tower_b200 import Cache
+    cfg = S.EncoderConfig(name="cache", n_mels=80, d_model=256, n_layers=2, n_heads=4, ffn_dim=512, frames=300,
+                          batch=4, dtype="bf16", seed=21)
+    enc = make_encoder(cfg, to_device(cfg, S.make_weights(cfg)))
+    mel = torch.from_numpy(S.make_mel(cfg.replace(batch=6))).to(device="cuda", dtype=torch.bfloat16)
+    return cfg, enc, mel, Cache(enc, capacity)
+
+
+def test_hits_equal_fresh_forward_bit_for_bit():
+    import torch
+    cfg, enc, mel, cache = _setup(8)
+    lengths = np.array([300, 201, 77, 300, 150, 9], np.int32)
+    sel = [0, 1, 2]
+    out, hits = cache.forward(mel[sel].contiguous(), keys=[10, 11, 12], lengths=lengths[sel])
+    ref = enc.forward(mel[sel].contiguous(), lengths[sel])
+    torch.cuda.synchronize()
+    assert list(hits) == [0, 0, 0] and cache.size() == 3
+    assert torch.equal(out, ref)
+    sel = [1, 3, 0, 3]                                   # keys 11 and 10 hit; key 13 twice, computed once
+    out, hits = cache.forward(mel[sel].contiguous(), keys=[11, 13, 10, 13], lengths=lengths[sel])
+    ref = enc.forward(mel[sel].contiguous(), lengths[sel])
+    torch.cuda.synchronize()
+    assert list(hits) == [1, 0, 1, 0] and cache.size() == 4
+    assert torch.equal(out, ref)
+    enc.status()
+    cache.close()
+    enc.close()
+
+
+def test_least_recently_used_is_replaced():
+    import torch
+    cfg, enc, mel, cache = _setup(2)
+    one = lambda i, key: cache.forward(mel[i:i + 1].contiguous(), keys=[key])[1][0]   # noqa: E731
+    assert one(0, 1) == 0 and one(1, 2) == 0 and cache.size() == 2
+    assert one(0, 1) == 1                                # key 1 used last: key 2 is now the oldest
+    assert one(2, 3) == 0 and cache.size() == 2          # replaces key 2
+    assert one(0, 1) == 1 and one(1, 2) == 0             # key 2 was dropped, key 1 kept
+    out, _ = cache.forward(mel[2:3].contiguous(), keys=[3])   # key 3 was replaced by key 2 just now
+    ref = enc.forward(mel[2:3].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    enc.status()
+    cache.close()
+    enc.close()
+
+
+def test_argument_errors():
+    from audio_encoder_tower_b200 import Cache, EncError
+    cfg, enc, mel, cache = _setup(2)
+    with pytest.raises(EncError):
+        cache.forward(mel[:5].contiguous(), keys=[1, 2, 3, 4, 5])          # B > max_batch
+    with pytest.raises(EncError):
+        cache.forward(mel[:1].contiguous(), keys=[1], lengths=[301])       # length > T
+    with pytest.raises(EncError):
+        Cache(enc, 0)
+    cache.close()
+    enc.close()
