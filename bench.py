@@ -213,6 +213,34 @@ def gemm_traffic_record():
     return rec if rec.get("source_sha256") == h.hexdigest() else None
 
 
+# ------------------------------------------------------------ multi-rank
+def rank_config(cfg, rank: int):
+    """The clips of one rank: the same weights (weight draws do not depend on the
+    seed offset of the inputs) and its own mel / lengths (seed + 1000 * rank)."""
+    return cfg.replace(seed=cfg.seed + 1000 * rank) if rank else cfg
+
+
+def rank_weight_seed(cfg) -> int:
+    """Every rank draws the weights from the unshifted seed."""
+    return cfg.seed
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The slowest rank's time: all-reduce MAX over the process group (any backend)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, audio_s_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job audio-seconds per second: every rank processes its own batch in the step time."""
+    return world * audio_s_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------- one kernel alone
 def run_kernel(args, cfg):
     """Time one step of the workload alone through the C ABI (for profiling): a
@@ -328,19 +356,12 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---- synthetic inputs and weights (per rank: own clips, same weights)
-    w_np = S.make_weights(cfg)
+    w_np = S.make_weights(cfg.replace(seed=rank_weight_seed(cfg)))
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     w_dev = {k: torch.from_numpy(v).to(device=dev, dtype=dt) for k, v in w_np.items()}
     del w_np
-    rcfg = cfg.replace(seed=cfg.seed + 1000 * rank) if rank else cfg
+    rcfg = rank_config(cfg, rank)
     lengths = S.make_lengths(rcfg)
     mel_np = S.make_mel(rcfg)
     enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
@@ -376,7 +397,7 @@ def main():
     launches = enc.launch_count() - n0
     clocks.stop()
     enc.status(stream)
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
 
     # ---- per-kernel-class breakdown: the same steps again with the library's
     # CUDA-event profiler on (kept out of the headline timing above)
@@ -437,7 +458,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     enc.status(stream)
     if not np.all(np.isfinite(out_host[last][0, :10].float().numpy())):
         raise RuntimeError("non-finite encoder output")
@@ -462,7 +483,7 @@ def main():
                    "share": v[0] / step_ms_prof} for k, v in prof.items()}
 
     tflops = flops / ms / 1e9
-    line = {"metric": METRIC, "value": world * audio_s / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+    line = {"metric": METRIC, "value": job_throughput(world, audio_s, ms), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; random weights)",
             "config": workload_desc(cfg, world),
@@ -472,7 +493,7 @@ def main():
             "peaks": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
             "roofline": roofline,
             "kernels": kernels,
-            "e2e": {"value": world * audio_s / (ms_e2e / 1e3), "unit": UNIT,
+            "e2e": {"value": job_throughput(world, audio_s, ms_e2e), "unit": UNIT,
                     "h2d_bytes_per_step": int(mel_host.numel() * mel_host.element_size()),
                     "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
                     "ms_per_step": ms_e2e,
