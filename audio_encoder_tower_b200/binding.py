@@ -23,7 +23,8 @@ EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status
             "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
             "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch",
             "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy",
-            "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy"]
+            "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy",
+            "enc_clip_flops", "enc_shard_plan"]
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -115,6 +116,11 @@ def load_library(path: str = LIB_PATH):
     lib.enc_cache_size.restype = ctypes.c_int32
     lib.enc_cache_destroy.argtypes = [_VP]
     lib.enc_cache_destroy.restype = None
+    lib.enc_clip_flops.argtypes = [ctypes.POINTER(EncConfig), ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]
+    lib.enc_clip_flops.restype = ctypes.c_int
+    lib.enc_shard_plan.argtypes = [ctypes.POINTER(EncConfig), i32p, ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p,
+                                   ctypes.POINTER(ctypes.c_double)]
+    lib.enc_shard_plan.restype = ctypes.c_int
     _LIB = lib
     return lib
 
@@ -139,6 +145,44 @@ def _stream_handle(stream) -> int | None:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def encoder_config(*, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
+                   pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0) -> EncConfig:
+    """The enc_config struct of a tower geometry (dtype "bf16" or "fp32")."""
+    return EncConfig(n_mels, d_model, n_layers, n_heads, head_dim, ffn_dim, max_frames, max_batch, pool_step,
+                     proj_hidden, proj_out, ln_eps, ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0,
+                     attn_chunk)
+
+
+def clip_flops(cfg: EncConfig, length: int) -> float:
+    """Algorithmic FLOPs of one clip of `length` valid frames (enc_clip_flops)."""
+    v = ctypes.c_double()
+    _check(load_library().enc_clip_flops(ctypes.byref(cfg), int(length), ctypes.byref(v)), "enc_clip_flops")
+    return float(v.value)
+
+
+def shard_plan(cfg: EncConfig, lengths, world: int):
+    """Split clips over `world` ranks of cfg.max_batch clips each (enc_shard_plan).
+
+    lengths: [B] valid frames per clip, or an int B for B full-length clips.
+    Returns (rank_of [B], index_of [B], rank_count [world], rank_flops [world]).
+    """
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    if isinstance(lengths, (int, np.integer)):
+        B, ln = int(lengths), None
+    else:
+        ln = np.ascontiguousarray(np.asarray(lengths, dtype=np.int32))
+        B = int(ln.shape[0])
+    rank_of = np.zeros(B, np.int32)
+    index_of = np.zeros(B, np.int32)
+    count = np.zeros(max(int(world), 1), np.int32)
+    flops = np.zeros(max(int(world), 1), np.float64)
+    _check(load_library().enc_shard_plan(ctypes.byref(cfg), None if ln is None else ln.ctypes.data_as(i32p), B,
+                                         int(world), rank_of.ctypes.data_as(i32p), index_of.ctypes.data_as(i32p),
+                                         count.ctypes.data_as(i32p),
+                                         flops.ctypes.data_as(ctypes.POINTER(ctypes.c_double))), "enc_shard_plan")
+    return rank_of, index_of, count, flops
+
+
 class Encoder:
     """One encoder handle (enc_create / enc_forward / enc_destroy).
 
@@ -150,9 +194,10 @@ class Encoder:
     def __init__(self, *, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
                  pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0, weights: dict):
         self.lib = load_library()
-        self.cfg = EncConfig(n_mels, d_model, n_layers, n_heads, head_dim, ffn_dim, max_frames, max_batch,
-                             pool_step, proj_hidden, proj_out, ln_eps,
-                             ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0, attn_chunk)
+        self.cfg = encoder_config(n_mels=n_mels, d_model=d_model, n_layers=n_layers, n_heads=n_heads,
+                                  ffn_dim=ffn_dim, max_frames=max_frames, max_batch=max_batch, dtype=dtype,
+                                  pool_step=pool_step, proj_hidden=proj_hidden, proj_out=proj_out, ln_eps=ln_eps,
+                                  head_dim=head_dim, attn_chunk=attn_chunk)
         w = EncWeights()
         for f in ("conv1_w", "conv1_b", "conv2_w", "conv2_b", "lnpost_g", "lnpost_b",
                   "proj1_w", "proj1_b", "proj2_w", "proj2_b"):

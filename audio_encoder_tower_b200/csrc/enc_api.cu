@@ -120,7 +120,9 @@ void free_all(enc_handle* h) {
   h->event_pool.clear();
 }
 
-enc_status validate_config(const enc_config* c) {
+}  // namespace
+
+enc_status enc::validate_config(const enc_config* c) {
   if (!c) return ENC_ERR_INVALID_ARG;
   if (c->flags != 0) return ENC_ERR_INVALID_ARG;
   if (c->dtype != ENC_DTYPE_BF16 && c->dtype != ENC_DTYPE_FP32) return ENC_ERR_INVALID_ARG;
@@ -147,6 +149,8 @@ enc_status validate_config(const enc_config* c) {
     return ENC_ERR_UNSUPPORTED;
   return ENC_OK;
 }
+
+namespace {
 
 // Copy `n` elements (cfg dtype) device to device into fresh library memory.
 enc_status copy_weight(enc_handle* h, const void* src, size_t n, void** dst) {

@@ -10,6 +10,9 @@
 
 namespace enc {
 
+// Geometry checks of enc_create, without the device check (host only).
+enc_status validate_config(const enc_config* c);
+
 // ----------------------------------------------------------- tcgen05 GEMM
 enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2 };
 

@@ -68,7 +68,8 @@ def workload_desc(cfg, n_gpus):
         "global_batch": cfg.batch * n_gpus,
         "frames": cfg.frames,
         "positions": cfg.positions,
-        "parallelism": f"replicas x{n_gpus} (batch sharded, no collective)",
+        "parallelism": (f"replicas x{n_gpus} (global batch of {cfg.batch * n_gpus} clips split by the cost-balanced "
+                        f"shard plan, {cfg.batch} per GPU; no collective)" if n_gpus > 1 else "replicas x1"),
         "l2": "per-step working set >> 126 MB L2 (weights 1.27 GB bf16 + activations), no explicit flush",
     }
 
@@ -214,10 +215,38 @@ def gemm_traffic_record():
 
 
 # ------------------------------------------------------------ multi-rank
-def rank_config(cfg, rank: int):
-    """The clips of one rank: the same weights (weight draws do not depend on the
-    seed offset of the inputs) and its own mel / lengths (seed + 1000 * rank)."""
-    return cfg.replace(seed=cfg.seed + 1000 * rank) if rank else cfg
+def tower_config(cfg, max_batch=None):
+    """The library's enc_config for a workload (max_batch = clips per rank)."""
+    from audio_encoder_tower_b200 import encoder_config
+    return encoder_config(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
+                          ffn_dim=cfg.ffn_dim, max_frames=cfg.frames,
+                          max_batch=cfg.batch if max_batch is None else max_batch, dtype=cfg.dtype,
+                          pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
+                          attn_chunk=cfg.attn_chunk)
+
+
+def rank_clips(cfg, rank: int, world: int):
+    """The clips of one rank: one seeded global batch of world x cfg.batch clips
+    (its first cfg.batch clips are the one-GPU batch) split over the ranks by the
+    library's cost-balanced plan (enc_shard_plan: largest clip first onto the
+    least loaded rank, cfg.batch clips per rank). Every rank computes the same
+    plan from the same lengths, so no rank sends it to another.
+    Returns (global-batch config, clip indices of this rank, their lengths)."""
+    g = cfg.replace(batch=cfg.batch * world)
+    lengths = S.make_lengths(g)
+    if world == 1:
+        return g, np.arange(cfg.batch), lengths
+    from audio_encoder_tower_b200 import shard_plan
+    rank_of, _, _, _ = shard_plan(tower_config(cfg), lengths, world)
+    mine = np.flatnonzero(rank_of == rank)     # clip order, as the plan's index_of
+    return g, mine, lengths[mine]
+
+
+def rank_mel(g, clips):
+    """The mel of the given clips of global-batch config g, [len(clips), n_mels, T]."""
+    if len(clips) == g.batch:
+        return S.make_mel(g)
+    return np.stack([S.mel_clip(g, int(b)) for b in clips])
 
 
 def rank_weight_seed(cfg) -> int:
@@ -236,9 +265,20 @@ def max_over_ranks(v: float, world: int, device) -> float:
     return float(t.item())
 
 
-def job_throughput(world: int, audio_s_per_rank: float, ms_per_step: float) -> float:
-    """Whole-job audio-seconds per second: every rank processes its own batch in the step time."""
-    return world * audio_s_per_rank / (ms_per_step / 1e3)
+def sum_over_ranks(v: float, world: int, device) -> float:
+    """A per-rank amount summed over the process group (any backend)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(audio_s_all_ranks: float, ms_per_step: float) -> float:
+    """Whole-job audio-seconds per second: the audio of every rank's batch in the slowest rank's step time."""
+    return audio_s_all_ranks / (ms_per_step / 1e3)
 
 
 # ------------------------------------------------------- one kernel alone
@@ -361,9 +401,8 @@ def main():
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     w_dev = {k: torch.from_numpy(v).to(device=dev, dtype=dt) for k, v in w_np.items()}
     del w_np
-    rcfg = rank_config(cfg, rank)
-    lengths = S.make_lengths(rcfg)
-    mel_np = S.make_mel(rcfg)
+    gcfg, clips, lengths = rank_clips(cfg, rank, world)
+    mel_np = rank_mel(gcfg, clips)
     enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
                   ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=cfg.batch, dtype=cfg.dtype,
                   pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
@@ -376,6 +415,8 @@ def main():
     stream = torch.cuda.current_stream(dev)
     audio_s = float(np.sum(lengths)) / FRAMES_PER_SECOND
     flops = workload_flops(cfg, lengths)
+    audio_s_job = sum_over_ranks(audio_s, world, dev)     # ragged clips: ranks differ in audio, not in cost
+    flops_job = sum_over_ranks(flops, world, dev)
 
     # ---- device-resident timing (inputs in HBM when the region starts)
     for _ in range(args.warmup):
@@ -482,8 +523,8 @@ def main():
     kernels = {k: {"ms_per_step": v[0] / args.steps, "tflops": (v[1] / v[0] / 1e9 if v[0] and v[1] else None),
                    "share": v[0] / step_ms_prof} for k, v in prof.items()}
 
-    tflops = flops / ms / 1e9
-    line = {"metric": METRIC, "value": job_throughput(world, audio_s, ms), "unit": UNIT, "n_gpus": world,
+    tflops = flops_job / world / ms / 1e9     # per GPU
+    line = {"metric": METRIC, "value": job_throughput(audio_s_job, ms), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; random weights)",
             "config": workload_desc(cfg, world),
@@ -493,7 +534,7 @@ def main():
             "peaks": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
             "roofline": roofline,
             "kernels": kernels,
-            "e2e": {"value": job_throughput(world, audio_s, ms_e2e), "unit": UNIT,
+            "e2e": {"value": job_throughput(audio_s_job, ms_e2e), "unit": UNIT,
                     "h2d_bytes_per_step": int(mel_host.numel() * mel_host.element_size()),
                     "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
                     "ms_per_step": ms_e2e,
