@@ -24,7 +24,7 @@ EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status
             "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch",
             "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy",
             "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy",
-            "enc_clip_flops", "enc_shard_plan"]
+            "enc_clip_flops", "enc_shard_plan", "enc_selftest_timeout"]
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -116,6 +116,8 @@ def load_library(path: str = LIB_PATH):
     lib.enc_cache_size.restype = ctypes.c_int32
     lib.enc_cache_destroy.argtypes = [_VP]
     lib.enc_cache_destroy.restype = None
+    lib.enc_selftest_timeout.argtypes = [_VP, ctypes.c_int64, _VP]
+    lib.enc_selftest_timeout.restype = ctypes.c_int
     lib.enc_clip_flops.argtypes = [ctypes.POINTER(EncConfig), ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]
     lib.enc_clip_flops.restype = ctypes.c_int
     lib.enc_shard_plan.argtypes = [ctypes.POINTER(EncConfig), i32p, ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p,
@@ -270,6 +272,12 @@ class Encoder:
     def status(self, stream=None):
         """Synchronise `stream` and raise if a device-side check or wait failed."""
         _check(self.lib.enc_get_status(self.handle, _stream_handle(stream)), "enc_get_status")
+
+    def selftest_timeout(self, limit_ns: int, stream=None):
+        """Enqueue the failure-detection self-test (enc_selftest_timeout): a bounded
+        wait that runs out after limit_ns; the next status() raises ENC_ERR_TIMEOUT."""
+        _check(self.lib.enc_selftest_timeout(self.handle, int(limit_ns), _stream_handle(stream)),
+               "enc_selftest_timeout")
 
     def profile(self, enable: bool):
         """Bracket every kernel of the following forwards with CUDA events."""

@@ -538,6 +538,33 @@ enc_status forward_f32(enc_handle* h, const void* mel, void* out, const Work& wk
 
 int valid_out(const enc_handle* h, int n) { return h->cfg.pool_step > 1 ? n / h->cfg.pool_step : n; }
 
+constexpr uint64_t kSelftestOtherNs = 2000000000ull;   // warp 1's own limit: 2 s
+
+// Failure detection without a fault (enc_selftest_timeout): two mbarrier
+// phases that nothing completes. Warp 0 gives up after limit_ns and raises
+// the abort flag; warp 1 leaves at its next check of the flag.
+__global__ void __launch_bounds__(64) selftest_timeout_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort_v = &abort_flag;
+  if (warp == 0) {
+    if (!mbar_wait_warp(&bars[0], 0, abort_v, limit_ns) && lane == 0) {
+      set_status(status, kDevTimeout);
+      *abort_v = 1;
+    }
+  } else {
+    mbar_wait_warp(&bars[1], 0, abort_v, kSelftestOtherNs);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -634,6 +661,13 @@ enc_status enc_get_status(enc_handle* h, cudaStream_t stream) {
   if (v == kDevTimeout) return ENC_ERR_TIMEOUT;
   if (v == kDevCheck) return ENC_ERR_DEVICE_CHECK;
   return v == 0 ? ENC_OK : ENC_ERR_CUDA;
+}
+
+enc_status enc_selftest_timeout(enc_handle* h, int64_t limit_ns, cudaStream_t stream) {
+  if (!h || limit_ns < 1000 || limit_ns > 100000000) return ENC_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 64, 0, stream>>>(h->status, static_cast<uint64_t>(limit_ns));
+  return cuda_status(cudaGetLastError());
 }
 
 void enc_destroy(enc_handle* h) {

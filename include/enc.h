@@ -162,6 +162,20 @@ ENC_API enc_status enc_output_positions(const enc_handle *h, int32_t B, const in
 /* Wait for `stream`, then read and clear the device status word of the handle. */
 ENC_API enc_status enc_get_status(enc_handle *h, cudaStream_t stream);
 
+/*
+ * Self-test of the device-side failure detection, without a fault: one CTA of
+ * two warps on `stream`. Warp 0 waits on an mbarrier phase that nothing
+ * completes, with the bounded wait of the GEMM and attention kernels, gives up
+ * after limit_ns, records ENC_ERR_TIMEOUT in the handle's status word and
+ * raises the CTA's abort flag; warp 1, waiting on a second such phase with a
+ * 2 s limit, leaves at its next check of that flag (the path every other warp
+ * of a failing CTA takes). Nothing traps and the context stays usable: the
+ * next enc_get_status returns ENC_ERR_TIMEOUT and clears the word, and later
+ * forwards run normally. Asynchronous.
+ *   limit_ns  1,000 .. 100,000,000 (1 us .. 100 ms), else ENC_ERR_INVALID_ARG
+ */
+ENC_API enc_status enc_selftest_timeout(enc_handle *h, int64_t limit_ns, cudaStream_t stream);
+
 /* Free everything the handle owns. Synchronises the device first. NULL is a no-op. */
 ENC_API void enc_destroy(enc_handle *h);
 

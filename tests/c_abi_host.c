@@ -59,6 +59,7 @@ int main(void) {
   cfg = tiny(4);
   check(enc_create(&cfg, &w, NULL) == ENC_ERR_INVALID_ARG, "enc_create without an output pointer");
   check(enc_forward(NULL, NULL, NULL, 1, NULL, NULL) == ENC_ERR_INVALID_ARG, "enc_forward without a handle");
+  check(enc_selftest_timeout(NULL, 1000000, NULL) == ENC_ERR_INVALID_ARG, "enc_selftest_timeout without a handle");
   enc_destroy(NULL);
   enc_cache_destroy(NULL);
   enc_frontend_destroy(NULL);

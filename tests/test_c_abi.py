@@ -25,4 +25,4 @@ def test_c_program_links_and_runs(tmp_path):
     lines = r.stdout.strip().splitlines()
     assert r.returncode == 0, r.stdout + r.stderr
     assert lines[-1] == "0 failures"
-    assert sum(1 for ln in lines if ln.startswith("ok ")) == 15
+    assert sum(1 for ln in lines if ln.startswith("ok ")) == 16
