@@ -513,7 +513,8 @@ def main():
     peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     ach = (g_fl / g_n) / (g_ms / g_n) / 1e9 if g_n else 0.0
     traffic = gemm_traffic_record()
-    roofline = {"kernel": "gemm_tc_kernel (tcgen05, all GEMM launches of the timed region)",
+    roofline = {"kernel": ("tcgen05 GEMM: gemm_tc2_kernel on SM pairs where N % 256 == 0 (every GEMM of the "
+                           "Whisper workloads), else gemm_tc_kernel; all GEMM launches of the timed region"),
                 "bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
                 "frac_of_burst_peak": ach / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
