@@ -166,3 +166,26 @@ def test_argument_errors():
     assert lib.enc_shard_plan(ctypes.byref(cfg), None, 9, 2, out.ctypes.data_as(i32p), None, None,
                               None) == ENC_ERR_INVALID_ARG
     assert (out == -7).all()
+
+
+def test_plan_properties_on_random_batches():
+    hyp = pytest.importorskip("hypothesis")
+    st = pytest.importorskip("hypothesis.strategies")
+
+    @hyp.settings(max_examples=150, deadline=None, derandomize=True)
+    @hyp.given(world=st.integers(1, 9), cap=st.integers(1, 12), data=st.data())
+    def check(world, cap, data):
+        B = data.draw(st.integers(1, world * cap))
+        lengths = np.array(data.draw(st.lists(st.integers(1, 40), min_size=B, max_size=B)), np.int32)
+        cfg = cfg_of(TINY, cap)
+        rank_of, index_of, count, flops = shard_plan(cfg, lengths, world)
+        _check_plan(lengths, world, cap, rank_of, index_of, count, flops, cfg)
+        # without a binding capacity (max_batch >= B) every clip goes onto the rank that
+        # is least loaded at that moment, so the most loaded rank ends at most the cost
+        # of its last clip above the final minimum
+        free = cfg_of(TINY, B)
+        _, _, _, f_free = shard_plan(free, lengths, world)
+        costs = np.array([clip_flops(free, int(x)) for x in lengths])
+        assert f_free.max() - f_free.min() <= costs.max() * (1 + 1e-12)
+
+    check()
