@@ -63,7 +63,8 @@ typedef enum enc_status {
   ENC_ERR_OOM = 3,           /* device or pinned allocation failed */
   ENC_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
   ENC_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out (status word) */
-  ENC_ERR_DEVICE_CHECK = 6   /* a device-side range check failed (status word) */
+  ENC_ERR_DEVICE_CHECK = 6   /* reserved for a device-side range check (status word); the host
+                                validates every input the kernels index by, so no kernel sets it */
 } enc_status;
 
 typedef enum enc_dtype {
