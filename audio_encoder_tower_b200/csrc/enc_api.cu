@@ -34,6 +34,11 @@ struct enc_handle {
   // allocations (all library-owned)
   std::vector<void*> allocs;
   size_t bytes = 0;
+  int alloc_calls = 0;       // device allocations attempted (ENC_FAIL_ALLOC test hook)
+  // enc_forward_static_scratch: device address of the library's static workspace
+  // on this handle's device, resolved in enc_create (nullptr when that failed)
+  unsigned char* static_scratch = nullptr;
+  enc_status static_scratch_status = ENC_ERR_CUDA;
   // repacked weights
   void* conv1_w = nullptr;   // [d, 3, mpad] (bf16) or [d, 3, n_mels] (fp32)
   void* conv2_w = nullptr;   // [d, 3, d]
@@ -86,10 +91,11 @@ template <typename P>
 enc_status dev_alloc(enc_handle* h, P** out, size_t bytes) {
   void* p = nullptr;
   if (bytes == 0) bytes = 16;
-  // Test hook: ENC_FAIL_ALLOC=N makes the N-th allocation (1-based) report failure.
-  static int counter = 0;
+  // Test hook: ENC_FAIL_ALLOC=N makes the handle's N-th device allocation (1-based,
+  // counted per handle, so every enc_create starts again at 1) report failure.
+  ++h->alloc_calls;
   const char* env = getenv("ENC_FAIL_ALLOC");
-  if (env && atoi(env) > 0 && ++counter == atoi(env)) return ENC_ERR_OOM;
+  if (env && atoi(env) > 0 && h->alloc_calls == atoi(env)) return ENC_ERR_OOM;
   cudaError_t e = cudaMalloc(&p, bytes);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -608,6 +614,7 @@ enc_status enc_create(const enc_config* cfg, const enc_weights* w, enc_handle** 
   h->p_out = cfg->pool_step > 1 ? h->P / cfg->pool_step : h->P;
   h->d_out = cfg->proj_hidden ? cfg->proj_out : cfg->d_model;
   st = build(h, w);
+  if (st == ENC_OK) resolve_static_scratch(h);
   if (st != ENC_OK) {
     cudaDeviceSynchronize();
     cudaGetLastError();
@@ -726,28 +733,27 @@ static __device__ __align__(256) unsigned char enc_static_scratch[ENC_STATIC_SCR
 
 namespace {
 
-void* g_static_scratch_base[64] = {};   // device address of enc_static_scratch, per device ordinal
-
-// Set-up, once per device, with that device current: the array's name is only a
-// host-side stand-in, so ask the runtime for its device address.
-enc_status static_scratch_base(int dev, unsigned char** base) {
-  if (dev < 0 || dev >= 64) return ENC_ERR_UNSUPPORTED;
-  if (!g_static_scratch_base[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, enc_static_scratch);
-    if (e != cudaSuccess || !p) {
-      cudaGetLastError();
-      return ENC_ERR_CUDA;
-    }
-    g_static_scratch_base[dev] = p;
-  }
-  *base = reinterpret_cast<unsigned char*>(g_static_scratch_base[dev]);
-  return ENC_OK;
-}
-
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 }  // namespace
+
+// Set-up of enc_forward_static_scratch, run by enc_create with the handle's
+// device current. In host code the array's name only stands in for it, so the
+// runtime is asked for its device address. The first lookup on a device loads
+// this file's module there, which is when the 64 MiB are reserved: in
+// enc_create, not inside enc_forward_static_scratch.
+void enc::resolve_static_scratch(enc_handle* h) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, enc_static_scratch);
+  if (e == cudaSuccess && p) {
+    h->static_scratch = reinterpret_cast<unsigned char*>(p);
+    h->static_scratch_status = ENC_OK;
+  } else {
+    cudaGetLastError();
+    h->static_scratch = nullptr;
+    h->static_scratch_status = e == cudaErrorMemoryAllocation ? ENC_ERR_OOM : ENC_ERR_CUDA;
+  }
+}
 
 extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel, const int32_t* lengths, int32_t B,
                                                  void* out, cudaStream_t stream) {
@@ -760,9 +766,9 @@ extern "C" enc_status enc_forward_static_scratch(enc_handle* h, const void* mel,
   const enc_config& c = h->cfg;
   const int d = c.d_model, F = c.ffn_dim, M = c.n_mels;
   if (cudaSetDevice(h->device) != cudaSuccess) return ENC_ERR_CUDA;
-  unsigned char* base = nullptr;
-  enc_status st = static_scratch_base(h->device, &base);
-  if (st != ENC_OK) return st;
+  unsigned char* base = h->static_scratch;   // resolved by enc_create
+  if (!base) return h->static_scratch_status;
+  enc_status st = ENC_OK;
 
   // per-clip counts, written straight into the handle's pinned staging buffer
   if (h->meta_pending) ENC_TRY(cudaEventSynchronize(h->meta_free));

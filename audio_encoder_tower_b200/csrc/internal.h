@@ -12,6 +12,8 @@ namespace enc {
 
 // Geometry checks of enc_create, without the device check (host only).
 enc_status validate_config(const enc_config* c);
+// enc_forward_static_scratch set-up (enc_create): the static workspace's device address.
+void resolve_static_scratch(enc_handle* h);
 
 // ----------------------------------------------------------- tcgen05 GEMM
 enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2 };
@@ -23,6 +25,7 @@ struct GemmTcParams {
   int kb_seg;      // k-blocks per tap segment (conv modes)
   int tiles_n;     // filled by the launcher
   int num_tiles;   // filled by the launcher
+  int tail;        // SM-pair kernel: the last `tail` tiles run as two 256 x 128 halves (launcher)
   EpiParams epi;
   int* status;
 };

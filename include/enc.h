@@ -98,8 +98,9 @@ typedef struct enc_config {
  * Weight device pointers in PyTorch layouts, element type cfg.dtype.
  * Per-layer entries are HOST arrays of n_layers device pointers.
  * Any bias / LayerNorm beta may be NULL (read as zeros); a NULL gamma reads as ones.
- * k_b must be NULL or all zeros: the key projection carries no bias (a key bias
- * adds the same amount to every score of a query row and cancels in softmax).
+ * k_b is accepted and ignored (NULL is the usual value): the key projection runs
+ * without a bias, because a key bias adds q.k_b to every score of a query row,
+ * a per-row constant that softmax cancels exactly, so it cannot change the output.
  */
 typedef struct enc_weights {
   const void *conv1_w;   /* [d, n_mels, 3] */
@@ -123,6 +124,9 @@ typedef struct enc_handle enc_handle;
 
 /*
  * Create an encoder on the current CUDA device. Synchronous.
+ * Passage: Qwen2-Audio-7B-Instruct, "(1) AUDIO ENCODER" (the Whisper-large geometry
+ * and weight shapes, e.g. q_proj [1280, 1280]); MiniCPM-o-2.6, "(2) AUDIO" (the
+ * medium-sized geometry, audio_pool_step); Voxtral-Mini-3B-2507, "PROJECTOR".
  * Validates cfg (ENC_ERR_UNSUPPORTED for geometry or a device other than sm_100),
  * copies and repacks the weights into library-owned device memory (fused QKV,
  * tap-major conv kernels, fp32 biases, position table) and allocates the
@@ -133,6 +137,10 @@ ENC_API enc_status enc_create(const enc_config *cfg, const enc_weights *w, enc_h
 
 /*
  * Enqueue one forward pass on `stream`. Asynchronous: returns once enqueued.
+ * Passage: Qwen2-Audio-7B-Instruct, "(1) AUDIO ENCODER" (one bidirectional pass,
+ * 30 s -> 1500 positions); Voxtral-Mini-3B-2507, "Preprocessor" (3000 mel frames
+ * per 30 s at 16 kHz, hop 160); "REQUIRED KERNEL CLASS" (the encoder on a schedule
+ * of its own, separate from the decoder: the caller's stream).
  *   mel      device [B, n_mels, T], cfg.dtype. Frames t >= lengths[b] are treated
  *            as silence (zero) whatever they hold.
  *   lengths  HOST [B] valid frames per clip, each in [1, T]; NULL means all T.
@@ -153,6 +161,9 @@ ENC_API enc_status enc_forward(enc_handle *h, const void *mel, const int32_t *le
 
 /*
  * Output geometry for a batch, computed on the host (no device work).
+ * Passage: Voxtral-Mini-3B-2507, "Preprocessor" and Qwen2-Audio-7B-Instruct,
+ * "(1) AUDIO ENCODER" (3000 frames -> 1500 positions); MiniCPM-o-2.6, "(2) AUDIO"
+ * (pool step 2: about 750 tokens per 30 s).
  *   n_out  HOST [B] (may be NULL): valid output rows per clip
  *   p_out  (may be NULL): rows per clip in `out` (the row stride is p_out * d_out)
  *   d_out  (may be NULL): width of an output row
@@ -160,11 +171,17 @@ ENC_API enc_status enc_forward(enc_handle *h, const void *mel, const int32_t *le
 ENC_API enc_status enc_output_positions(const enc_handle *h, int32_t B, const int32_t *lengths,
                                 int32_t *n_out, int32_t *p_out, int32_t *d_out);
 
-/* Wait for `stream`, then read and clear the device status word of the handle. */
+/*
+ * Wait for `stream`, then read and clear the device status word of the handle.
+ * Returns ENC_ERR_TIMEOUT if a bounded device-side wait ran out since the last
+ * call. (No passage: the pages describe the encoder's arithmetic, not how a
+ * library reports device-side errors.)
+ */
 ENC_API enc_status enc_get_status(enc_handle *h, cudaStream_t stream);
 
 /*
- * Self-test of the device-side failure detection, without a fault: one CTA of
+ * Self-test of the device-side failure detection (no passage: a property of this
+ * library), without a fault: one CTA of
  * two warps on `stream`. Warp 0 waits on an mbarrier phase that nothing
  * completes, with the bounded wait of the GEMM and attention kernels, gives up
  * after limit_ns, records ENC_ERR_TIMEOUT in the handle's status word and
@@ -177,13 +194,14 @@ ENC_API enc_status enc_get_status(enc_handle *h, cudaStream_t stream);
  */
 ENC_API enc_status enc_selftest_timeout(enc_handle *h, int64_t limit_ns, cudaStream_t stream);
 
-/* Free everything the handle owns. Synchronises the device first. NULL is a no-op. */
+/* Free everything the handle owns. Synchronises the device first. NULL is a no-op.
+ * (Library resource management; no passage.) */
 ENC_API void enc_destroy(enc_handle *h);
 
-/* Static description of a status code. */
+/* Static description of a status code (no passage). */
 ENC_API const char *enc_status_string(enc_status s);
 
-/* Library-owned device bytes: repacked weights and workspace (for reporting). */
+/* Library-owned device bytes: repacked weights and workspace (for reporting; no passage). */
 ENC_API size_t enc_device_bytes(const enc_handle *h);
 
 /*
@@ -196,16 +214,19 @@ ENC_API size_t enc_device_bytes(const enc_handle *h);
  * Same arguments, output and errors as enc_forward, with the handle's weights.
  * The per-batch workspace (time-major mel, conv1 output, residual stream, LN,
  * QKV, attention and FFN buffers, projector buffers, clip offsets) is carved
- * out of one file-scope static device array of 64 MiB (67,108,864 bytes) that
- * the CUDA runtime reserves on every device that loads this library and keeps
- * until the process exits. The call itself allocates nothing (no cudaMalloc,
- * no cudaFree, no allocating library routine).
+ * out of one file-scope static device array of 64 MiB (67,108,864 bytes). The
+ * CUDA runtime reserves it on a device when the library's module holding it is
+ * loaded there, and keeps it until the process exits.
+ *   - Set-up: enc_create looks up the array's device address on its device
+ *     (cudaGetSymbolAddress, with that device current); that lookup loads the
+ *     module, so the 64 MiB are reserved inside enc_create. This call itself
+ *     allocates nothing, its first call included (no cudaMalloc, no cudaFree, no
+ *     allocating library routine). If the lookup failed in enc_create (too little
+ *     device memory left for the array), enc_create still succeeds and this call
+ *     returns ENC_ERR_OOM (ENC_ERR_CUDA for another runtime error).
  *   - Capacity: a batch whose workspace exceeds 64 MiB returns
  *     ENC_ERR_INVALID_ARG before anything is enqueued. One 30 s clip of the
  *     Whisper-large encoder (about 51 MB of workspace) fits; two do not.
- *   - Set-up: the first call on a device looks up the device address of the
- *     array (cudaGetSymbolAddress, with that device current). Make that first
- *     call before any stream capture.
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     previous call's contents; the call clears what it reads as zero. Calls
  *     whose GPU work overlaps (other streams, other handles, other threads)

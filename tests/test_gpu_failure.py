@@ -40,3 +40,40 @@ def test_timeout_is_reported_and_the_context_survives():
         assert ei.value.code == ENC_ERR_INVALID_ARG
     enc.status()
     enc.close()
+
+
+def test_allocation_failure_at_every_point_frees_everything(monkeypatch):
+    """ENC_FAIL_ALLOC=N makes the N-th device allocation of one enc_create report
+    failure: a host-side failure, no device fault. For every N up to the number of
+    allocations a handle makes, enc_create returns ENC_ERR_OOM and leaves nothing
+    allocated (the device's free memory is the same after the whole sweep); the
+    counter restarts with every enc_create, and without the hook creation works."""
+    import torch
+    from audio_encoder_tower_b200.binding import ENC_ERR_OOM
+    # a 30 s workspace, so that a leaked buffer would show in the free memory
+    cfg = S.EncoderConfig(name="oom", n_mels=128, d_model=256, n_layers=2, n_heads=4, ffn_dim=1024, frames=3000,
+                          batch=2, dtype="bf16", seed=14)
+    w = to_device(cfg, S.make_weights(cfg))
+    monkeypatch.delenv("ENC_FAIL_ALLOC", raising=False)
+    make_encoder(cfg, w).close()               # modules loaded, runtime pools warm
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    failed = 0
+    for n in range(1, 500):
+        monkeypatch.setenv("ENC_FAIL_ALLOC", str(n))
+        try:
+            enc = make_encoder(cfg, w)
+        except EncError as e:
+            assert e.code == ENC_ERR_OOM, (n, e.code)
+            failed += 1
+            continue
+        enc.close()                            # n is past the last allocation
+        break
+    else:
+        pytest.fail("enc_create never got past the hook")
+    monkeypatch.delenv("ENC_FAIL_ALLOC")
+    assert failed >= 30                        # weights, biases, workspace: every one was a failure point
+    torch.cuda.synchronize()
+    assert abs(torch.cuda.mem_get_info()[0] - free0) < (8 << 20)
+    enc = make_encoder(cfg, w)
+    enc.close()

@@ -61,15 +61,19 @@ def test_small_configs(cfg, lengths):
 
 def test_peaky_bf16():
     """Weights N(0, 0.2) (ten times the workloads' scale) make softmax peaky and
-    grow activations layer over layer; bf16 rounding at the GEMM operands then
-    gives about 1.6-1.9% relative Frobenius error (reproduced by emulating the
-    same rounding points in float64). Bound: 3e-2 / 0.3."""
+    grow activations layer over layer, so bf16 rounding alone moves the output by
+    1.5-1.9%: more than the workloads' 1e-2. The bound is that rounding's own
+    size on the same clip, from the rounding-point model (oracle/bf16_model.py):
+    relative Frobenius error <= 1.4x the model's + 2e-3, max-abs <= 2x the model's."""
+    from oracle.bf16_model import encode_clip_bf16
     cfg = _small("peaky", weight_std=0.2, frames=260)
     lengths = [260, 131, 65]
     w, mel, got, n_out, p_out, d_out = _run_case(cfg, np.array(lengths, np.int32))
     for b, ln in enumerate(lengths):
-        m = compare(cfg, got[b], oracle_clip(cfg, w, mel[b], ln), int(n_out[b]))
-        assert m["rel_fro"] <= 3e-2 and m["max_abs"] <= 0.3, m
+        ref = oracle_clip(cfg, w, mel[b], ln)
+        band = compare(cfg, encode_clip_bf16(cfg, w, mel[b], ln), ref, int(n_out[b]))
+        m = compare(cfg, got[b], ref, int(n_out[b]))
+        assert m["rel_fro"] <= 1.4 * band["rel_fro"] + 2e-3 and m["max_abs"] <= 2.0 * band["max_abs"], (m, band)
 
 
 def test_tiny_fp32_whole():
@@ -126,21 +130,29 @@ def test_argument_errors():
 
 
 # ------------------------------------------------------------- full sizes
-FULL = [("medium_pool", [0]), ("large_b16", [5]), ("large_proj_b32", [31]), ("large_ragged_b64", None),
-        ("large_pool4_b16", [3]), ("medium_chunk50", [2])]
+# (workload, sampled clips, clip checked alone against its slot in the batch)
+FULL = [("medium_pool", [0], None), ("large_b16", [5], 5), ("large_proj_b32", [31], None),
+        ("large_ragged_b64", None, None), ("large_pool4_b16", [3], None), ("medium_chunk50", [2], None)]
 
 
-@pytest.mark.parametrize("name,sample", FULL, ids=[n for n, _ in FULL])
-def test_full_size_sampled(name, sample):
+@pytest.mark.parametrize("name,sample,alone", FULL, ids=[n for n, _, _ in FULL])
+def test_full_size_sampled(name, sample, alone):
     cfg = S.CONFIGS[name]
     lengths = S.make_lengths(cfg)
-    if sample is None:                       # the ragged sweep: its shortest and longest clip
-        sample = [int(np.argmin(lengths)), int(np.argmax(lengths))]
+    if sample is None:   # the ragged sweep: its shortest and longest clip, and its first odd-length clip
+        odd = [b for b in range(cfg.batch) if lengths[b] % 2 == 1]
+        sample = sorted({int(np.argmin(lengths)), int(np.argmax(lengths)), odd[0]})
+        alone = odd[0]
     w = S.make_weights(cfg)
     mel = S.make_mel(cfg)
     enc = make_encoder(cfg, to_device(cfg, w))
     got = run_gpu(enc, cfg, mel, lengths)
     n_out, p_out, d_out = enc.output_positions(cfg.batch, lengths)
+    if alone is not None:
+        # at full size the GEMM tile grid and the attention grid differ between a
+        # batch and one clip: the clip's output must not (bit-exact)
+        one = run_gpu(enc, cfg, mel[alone:alone + 1], lengths[alone:alone + 1])
+        np.testing.assert_array_equal(one[0], got[alone])
     enc.close()
     assert got.shape == (cfg.batch, p_out, d_out)
     # shapes and padding masks, every clip (bit-exact)
