@@ -23,8 +23,10 @@ EXPORTED = ["enc_create", "enc_forward", "enc_output_positions", "enc_get_status
             "enc_status_string", "enc_device_bytes", "enc_linear_bf16", "enc_attention_bf16",
             "enc_profile_enable", "enc_profile_collect", "enc_launch_count", "enc_forward_static_scratch",
             "enc_frontend_create", "enc_frontend_log_mel", "enc_frontend_destroy",
-            "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy",
-            "enc_clip_flops", "enc_shard_plan", "enc_selftest_timeout"]
+            "enc_cache_create", "enc_forward_cached", "enc_cache_size", "enc_cache_destroy", "enc_cache_content_keys",
+            "enc_clip_flops", "enc_shard_plan", "enc_selftest_timeout", "enc_check_guards",
+            "enc_guard_selftest"]
+ENC_FLAG_GUARD = 1
 
 KERNEL_CLASSES = ["mel", "conv1", "conv2", "ln", "qkv", "attn", "out", "fc1", "fc2", "final", "proj1", "proj2",
                   "zero"]
@@ -112,10 +114,16 @@ def load_library(path: str = LIB_PATH):
     lib.enc_forward_cached.argtypes = [_VP, _VP, i32p, ctypes.POINTER(ctypes.c_uint64), ctypes.c_int32, _VP, i32p,
                                        _VP]
     lib.enc_forward_cached.restype = ctypes.c_int
+    lib.enc_cache_content_keys.argtypes = [_VP, _VP, i32p, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint64), _VP]
+    lib.enc_cache_content_keys.restype = ctypes.c_int
     lib.enc_cache_size.argtypes = [_VP]
     lib.enc_cache_size.restype = ctypes.c_int32
     lib.enc_cache_destroy.argtypes = [_VP]
     lib.enc_cache_destroy.restype = None
+    lib.enc_check_guards.argtypes = [_VP, ctypes.c_char_p, ctypes.c_size_t]
+    lib.enc_check_guards.restype = ctypes.c_int
+    lib.enc_guard_selftest.argtypes = [_VP, ctypes.c_int32, ctypes.c_int64]
+    lib.enc_guard_selftest.restype = ctypes.c_int
     lib.enc_selftest_timeout.argtypes = [_VP, ctypes.c_int64, _VP]
     lib.enc_selftest_timeout.restype = ctypes.c_int
     lib.enc_clip_flops.argtypes = [ctypes.POINTER(EncConfig), ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]
@@ -148,11 +156,12 @@ def _stream_handle(stream) -> int | None:
 
 
 def encoder_config(*, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
-                   pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0) -> EncConfig:
-    """The enc_config struct of a tower geometry (dtype "bf16" or "fp32")."""
+                   pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0,
+                   guard=False) -> EncConfig:
+    """The enc_config struct of a tower geometry (dtype "bf16" or "fp32"); guard sets ENC_FLAG_GUARD."""
     return EncConfig(n_mels, d_model, n_layers, n_heads, head_dim, ffn_dim, max_frames, max_batch, pool_step,
-                     proj_hidden, proj_out, ln_eps, ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32, 0,
-                     attn_chunk)
+                     proj_hidden, proj_out, ln_eps, ENC_DTYPE_BF16 if dtype == "bf16" else ENC_DTYPE_FP32,
+                     ENC_FLAG_GUARD if guard else 0, attn_chunk)
 
 
 def clip_flops(cfg: EncConfig, length: int) -> float:
@@ -194,12 +203,13 @@ class Encoder:
     """
 
     def __init__(self, *, n_mels, d_model, n_layers, n_heads, ffn_dim, max_frames, max_batch, dtype="bf16",
-                 pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0, weights: dict):
+                 pool_step=1, proj_hidden=0, proj_out=0, ln_eps=1e-5, head_dim=64, attn_chunk=0, guard=False,
+                 weights: dict):
         self.lib = load_library()
         self.cfg = encoder_config(n_mels=n_mels, d_model=d_model, n_layers=n_layers, n_heads=n_heads,
                                   ffn_dim=ffn_dim, max_frames=max_frames, max_batch=max_batch, dtype=dtype,
                                   pool_step=pool_step, proj_hidden=proj_hidden, proj_out=proj_out, ln_eps=ln_eps,
-                                  head_dim=head_dim, attn_chunk=attn_chunk)
+                                  head_dim=head_dim, attn_chunk=attn_chunk, guard=guard)
         w = EncWeights()
         for f in ("conv1_w", "conv1_b", "conv2_w", "conv2_b", "lnpost_g", "lnpost_b",
                   "proj1_w", "proj1_b", "proj2_w", "proj2_b"):
@@ -272,6 +282,18 @@ class Encoder:
     def status(self, stream=None):
         """Synchronise `stream` and raise if a device-side check or wait failed."""
         _check(self.lib.enc_get_status(self.handle, _stream_handle(stream)), "enc_get_status")
+
+    def check_guards(self):
+        """enc_check_guards (handles created with guard=True): raise EncError naming the
+        buffer and offset if a kernel wrote into a guard region around a workspace buffer."""
+        msg = ctypes.create_string_buffer(256)
+        code = self.lib.enc_check_guards(self.handle, msg, 256)
+        if code != ENC_OK:
+            raise EncError(code, "enc_check_guards: " + msg.value.decode())
+
+    def guard_selftest(self, buffer: int, offset: int):
+        """enc_guard_selftest: one guard byte changed from the host is reported, then restored."""
+        _check(self.lib.enc_guard_selftest(self.handle, int(buffer), int(offset)), "enc_guard_selftest")
 
     def selftest_timeout(self, limit_ns: int, stream=None):
         """Enqueue the failure-detection self-test (enc_selftest_timeout): a bounded
@@ -382,10 +404,25 @@ class Cache:
         _check(self.lib.enc_cache_create(encoder.handle, int(capacity), ctypes.byref(h)), "enc_cache_create")
         self.h = h
 
-    def forward(self, mel, keys, lengths=None, out=None, stream=None):
-        """Returns (out, hits): hits[b] = 1 where clip b's output came from the cache."""
+    def content_keys(self, mel, lengths=None, stream=None) -> np.ndarray:
+        """enc_cache_content_keys: [B] uint64 keys hashed from each clip's length and
+        valid mel frames on the device (waits for `stream`)."""
+        B = int(mel.shape[0])
+        ln = None if lengths is None else np.ascontiguousarray(np.asarray(lengths, dtype=np.int32))
+        keys = np.zeros(B, dtype=np.uint64)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        _check(self.lib.enc_cache_content_keys(self.h, _ptr(mel), None if ln is None else ln.ctypes.data_as(i32p),
+                                               B, keys.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64)),
+                                               _stream_handle(stream)), "enc_cache_content_keys")
+        return keys
+
+    def forward(self, mel, keys=None, lengths=None, out=None, stream=None):
+        """Returns (out, hits): hits[b] = 1 where clip b's output came from the cache.
+        keys=None derives each clip's key from its content (content_keys)."""
         import torch
         B = int(mel.shape[0])
+        if keys is None:
+            keys = self.content_keys(mel, lengths, stream)
         if out is None:
             _, p_out, d_out = self.encoder.output_positions(B, lengths)
             out = torch.empty((B, p_out, d_out), dtype=mel.dtype, device=mel.device)

@@ -6,6 +6,8 @@
 
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/enc.h"
 #include "../../include/enc_profile.h"
 #include "common.cuh"
@@ -35,6 +37,9 @@ struct enc_handle {
   std::vector<void*> allocs;
   size_t bytes = 0;
   int alloc_calls = 0;       // device allocations attempted (ENC_FAIL_ALLOC test hook)
+  // ENC_FLAG_GUARD: guard regions around every workspace buffer
+  struct Guard { const char* name; unsigned char* buf; size_t bytes; };
+  std::vector<Guard> guards;
   // enc_forward_static_scratch: device address of the library's static workspace
   // on this handle's device, resolved in enc_create (nullptr when that failed)
   unsigned char* static_scratch = nullptr;
@@ -113,6 +118,26 @@ enc_status dev_alloc(enc_handle* h, P** out, size_t bytes) {
     if (_s != ENC_OK) return _s;               \
   } while (0)
 
+constexpr size_t kGuardBytes = 256u << 10;   // each side of a guarded workspace buffer
+constexpr unsigned char kGuardByte = 0xA5;
+
+// A workspace buffer of the handle. With ENC_FLAG_GUARD it sits between two
+// guard regions of kGuardBytes filled with kGuardByte (the buffer keeps 256-byte
+// alignment); enc_check_guards reads them back.
+template <typename P>
+enc_status ws_alloc(enc_handle* h, P** out, size_t bytes, const char* name) {
+  if (!(h->cfg.flags & ENC_FLAG_GUARD)) return dev_alloc(h, out, bytes);
+  const size_t inner = (bytes + 255) & ~size_t(255);
+  unsigned char* base = nullptr;
+  ENC_CHECK(dev_alloc(h, &base, inner + 2 * kGuardBytes));
+  if (cudaMemset(base, kGuardByte, kGuardBytes) != cudaSuccess ||
+      cudaMemset(base + kGuardBytes + inner, kGuardByte, kGuardBytes) != cudaSuccess)
+    return ENC_ERR_CUDA;
+  h->guards.push_back({name, base + kGuardBytes, inner});
+  *out = reinterpret_cast<P*>(base + kGuardBytes);
+  return ENC_OK;
+}
+
 void free_all(enc_handle* h) {
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
@@ -130,7 +155,7 @@ void free_all(enc_handle* h) {
 
 enc_status enc::validate_config(const enc_config* c) {
   if (!c) return ENC_ERR_INVALID_ARG;
-  if (c->flags != 0) return ENC_ERR_INVALID_ARG;
+  if (c->flags & ~ENC_FLAG_GUARD) return ENC_ERR_INVALID_ARG;
   if (c->dtype != ENC_DTYPE_BF16 && c->dtype != ENC_DTYPE_FP32) return ENC_ERR_INVALID_ARG;
   if (c->n_mels <= 0 || c->d_model <= 0 || c->n_layers < 0 || c->n_heads <= 0 || c->ffn_dim <= 0 ||
       c->max_frames <= 0 || c->max_batch <= 0)
@@ -233,18 +258,18 @@ enc_status build(enc_handle* h, const enc_weights* w) {
   ENC_TRY(launch_position_table(h->pe, h->P, d, 0));
   // ---- workspace
   const long long rows_t = (long long)Bm * h->Tp, rows_p = (long long)Bm * h->P, rows_o = (long long)Bm * h->p_out;
-  ENC_CHECK(dev_alloc(h, &h->melT, (size_t)(rows_t + 2) * M * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->y1, (size_t)(rows_t + 2) * d * h->esz));
+  ENC_CHECK(ws_alloc(h, &h->melT, (size_t)(rows_t + 2) * M * h->esz, "melT"));
+  ENC_CHECK(ws_alloc(h, &h->y1, (size_t)(rows_t + 2) * d * h->esz, "y1"));
   ENC_TRY(cudaMemset(h->melT, 0, (size_t)(rows_t + 2) * M * h->esz));
   ENC_TRY(cudaMemset(h->y1, 0, (size_t)(rows_t + 2) * d * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->x, (size_t)rows_p * d * 4));
-  ENC_CHECK(dev_alloc(h, &h->a, (size_t)rows_p * d * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->qkv, (size_t)rows_p * 3 * d * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->o, (size_t)rows_p * d * h->esz));
-  ENC_CHECK(dev_alloc(h, &h->f, (size_t)rows_p * F * h->esz));
+  ENC_CHECK(ws_alloc(h, &h->x, (size_t)rows_p * d * 4, "x"));
+  ENC_CHECK(ws_alloc(h, &h->a, (size_t)rows_p * d * h->esz, "a"));
+  ENC_CHECK(ws_alloc(h, &h->qkv, (size_t)rows_p * 3 * d * h->esz, "qkv"));
+  ENC_CHECK(ws_alloc(h, &h->o, (size_t)rows_p * d * h->esz, "o"));
+  ENC_CHECK(ws_alloc(h, &h->f, (size_t)rows_p * F * h->esz, "f"));
   if (ph) {
-    ENC_CHECK(dev_alloc(h, &h->e, (size_t)rows_o * d * h->esz));
-    ENC_CHECK(dev_alloc(h, &h->p1, (size_t)rows_o * ph * h->esz));
+    ENC_CHECK(ws_alloc(h, &h->e, (size_t)rows_o * d * h->esz, "e"));
+    ENC_CHECK(ws_alloc(h, &h->p1, (size_t)rows_o * ph * h->esz, "p1"));
   }
   ENC_TRY(cudaMemset(h->x, 0, (size_t)rows_p * d * 4));
   ENC_TRY(cudaMemset(h->a, 0, (size_t)rows_p * d * h->esz));
@@ -253,8 +278,8 @@ enc_status build(enc_handle* h, const enc_weights* w) {
   ENC_TRY(cudaMemset(h->f, 0, (size_t)rows_p * F * h->esz));
   // block-local attention adds the chunk boundaries: at most ceil(P / chunk) per clip
   h->meta_ints = 3 * Bm + 2 + (c.attn_chunk > 0 ? Bm * ((h->P + c.attn_chunk - 1) / c.attn_chunk) + 1 : 0);
-  ENC_CHECK(dev_alloc(h, &h->meta, (size_t)h->meta_ints * 4));
-  ENC_CHECK(dev_alloc(h, &h->status, 4));
+  ENC_CHECK(ws_alloc(h, &h->meta, (size_t)h->meta_ints * 4, "meta"));
+  ENC_CHECK(ws_alloc(h, &h->status, 4, "status"));
   ENC_TRY(cudaMemset(h->status, 0, 4));
   if (cudaMallocHost(&h->h_meta, (size_t)h->meta_ints * 4) != cudaSuccess) {
     cudaGetLastError();
@@ -315,9 +340,23 @@ cudaEvent_t pooled_event(enc_handle* h) {
   return e;
 }
 
+// NVTX range names of the kernel classes (include/enc_profile.h order). The
+// ranges mark host-side enqueueing for a tool such as Nsight Systems; with no
+// tool attached each push / pop is a check of one pointer.
+const char* const kRangeNames[ENC_K_COUNT] = {"mel stage", "conv1", "conv2", "layernorm", "qkv", "attention",
+                                              "out-proj", "fc1", "fc2", "final layernorm", "projector fc1",
+                                              "projector fc2", "zero rows"};
+
+// RAII NVTX range
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
+
 // Enqueue one kernel: bracket it with events when profiling, count it.
 template <typename F>
 cudaError_t run(enc_handle* h, cudaStream_t s, int cls, double flops, F&& launch) {
+  Range range(cls >= 0 && cls < ENC_K_COUNT ? kRangeNames[cls] : "kernel");
   cudaEvent_t a = nullptr, b = nullptr;
   if (h->profile) {
     a = pooled_event(h);
@@ -420,6 +459,7 @@ enc_status forward_bf16(enc_handle* h, const void* mel, void* out, const Work& w
 
   bf16* a = reinterpret_cast<bf16*>(h->a);
   for (int l = 0; l < c.n_layers; ++l) {
+    Range block("encoder block");
     const LayerMaps& lm = h->lmaps[l];
     ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<bf16>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
     g.M = R; g.a_mode = A_PLAIN; g.kb_seg = 0;
@@ -499,6 +539,7 @@ enc_status forward_f32(enc_handle* h, const void* mel, void* out, const Work& wk
   float* o = reinterpret_cast<float*>(h->o);
   float* f = reinterpret_cast<float*>(h->f);
   for (int l = 0; l < c.n_layers; ++l) {
+    Range block("encoder block");
     ENC_RUN(ENC_K_LN, 0.0, launch_layernorm<float>(h->x, h->ln1_g[l], h->ln1_b[l], a, R, d, c.ln_eps, s));
     e = epi_base(EPI_STORE);
     e.bias = h->qkv_b[l]; e.out = qkv; e.ldo = 3 * d;
@@ -654,6 +695,7 @@ enc_status enc_forward(enc_handle* h, const void* mel, const int32_t* lengths, i
   ENC_TRY(cudaMemcpyAsync(h->meta, h->h_meta, (size_t)nints * 4, cudaMemcpyHostToDevice, stream));
   ENC_TRY(cudaEventRecord(h->meta_free, stream));
   h->meta_pending = true;
+  Range range("enc_forward");
   return h->bf16 ? forward_bf16(h, mel, out, wk, stream) : forward_f32(h, mel, out, wk, stream);
 }
 
@@ -686,6 +728,44 @@ void enc_destroy(enc_handle* h) {
 }
 
 size_t enc_device_bytes(const enc_handle* h) { return h ? h->bytes : 0; }
+
+enc_status enc_guard_selftest(enc_handle* h, int32_t buffer, int64_t offset) {
+  if (!h || !(h->cfg.flags & ENC_FLAG_GUARD) || buffer < 0 || buffer >= (int32_t)h->guards.size())
+    return ENC_ERR_INVALID_ARG;
+  const auto& g = h->guards[buffer];
+  if (offset == 0 || offset < -(int64_t)kGuardBytes || offset > (int64_t)kGuardBytes) return ENC_ERR_INVALID_ARG;
+  // offset < 0: byte -offset before the buffer; offset > 0: byte offset - 1 past its end
+  unsigned char* p = offset < 0 ? g.buf + offset : g.buf + g.bytes + (offset - 1);
+  if (cudaSetDevice(h->device) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return ENC_ERR_CUDA;
+  if (cudaMemset(p, kGuardByte ^ 0xFF, 1) != cudaSuccess) return ENC_ERR_CUDA;
+  char msg[128];
+  const enc_status seen = enc_check_guards(h, msg, sizeof msg);
+  if (cudaMemset(p, kGuardByte, 1) != cudaSuccess) return ENC_ERR_CUDA;
+  if (seen != ENC_ERR_DEVICE_CHECK || strncmp(msg, g.name, strlen(g.name)) != 0) return ENC_ERR_CUDA;
+  return enc_check_guards(h, nullptr, 0);
+}
+
+enc_status enc_check_guards(enc_handle* h, char* what, size_t what_len) {
+  if (!h) return ENC_ERR_INVALID_ARG;
+  if (what && what_len) what[0] = 0;
+  if (!(h->cfg.flags & ENC_FLAG_GUARD)) return ENC_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return ENC_ERR_CUDA;
+  std::vector<unsigned char> buf(kGuardBytes);
+  for (const auto& g : h->guards) {
+    for (int side = 0; side < 2; ++side) {
+      const unsigned char* src = side ? g.buf + g.bytes : g.buf - kGuardBytes;
+      if (cudaMemcpy(buf.data(), src, kGuardBytes, cudaMemcpyDeviceToHost) != cudaSuccess) return ENC_ERR_CUDA;
+      for (size_t i = 0; i < kGuardBytes; ++i) {
+        if (buf[i] == kGuardByte) continue;
+        if (what && what_len)
+          snprintf(what, what_len, "%s: byte %s%zu %s the buffer changed", g.name, side ? "+" : "-",
+                   side ? i : kGuardBytes - i, side ? "past the end of" : "before the start of");
+        return ENC_ERR_DEVICE_CHECK;
+      }
+    }
+  }
+  return ENC_OK;
+}
 
 enc_status enc_profile_enable(enc_handle* h, int32_t enable) {
   if (!h) return ENC_ERR_INVALID_ARG;

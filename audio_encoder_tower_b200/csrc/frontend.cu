@@ -1,4 +1,4 @@
-// Log-mel front end on the GPU (fp32, CUDA cores): 30 s of 16 kHz audio ->
+// Log-mel front end on the GPU: 30 s of 16 kHz audio ->
 // the encoder's [n_mels, 3000] input features. Geometry from the pages
 // (Voxtral-Mini-3B-2507, "Preprocessor": WhisperFeatureExtractor, 480,000
 // samples, hop 160, 3000 frames, 128 features; MiniCPM-o-2.6, "(2) AUDIO": 80);
@@ -8,10 +8,18 @@
 // Steps for B clips:
 //   1. pad_kernel: each clip reflected by 200 samples at both ends into rows of
 //      a buffer whose clip stride is 3003 frames x 160 samples, so frame f of
-//      clip b starts at sample (b * 3003 + f) * 160 for every clip
-//   2. SGEMM: overlapping 400-sample rows (row stride 160) x the windowed
-//      cos / sin basis -> X [B * 3003, 404] (real | imaginary parts)
-//   3. power_kernel: |X_k|^2 for the 201 bins
+//      clip b starts at sample (b * 3003 + f) * 160 for every clip. Each
+//      sample a is stored twice: a_hi = a rounded to tf32 in one plane, a_lo =
+//      a - a_hi (exact in fp32) in a second plane.
+//   2. tensor cores (kind::tf32): the windowed DFT of every frame and its power
+//      spectrum, P [B * 3003, 204] = |X_k|^2. The product of the frames with the
+//      windowed cos / sin basis runs as one GEMM over K = 3 x 416 of
+//      [a_hi | a_hi | a_lo] and [w_hi | w_lo | w_hi]: a_hi w_hi + a_hi w_lo +
+//      a_lo w_hi is the fp32 product to about 2^-22 relative (the a_lo w_lo term
+//      and the tf32 truncation of the remainders are what it leaves out), an
+//      error-compensated split of the fp32 operands into tf32 pairs. The basis
+//      interleaves cos and sin of each bin, so the epilogue finds both parts of
+//      a bin in adjacent accumulator columns.
 //   4. SGEMM: power x filterbank^T -> mel [B * 3003, n_mels]
 //   5. log_max_kernel: log10(max(mel, 1e-10)) in place over the 3000 frames
 //      kept, and the clip's maximum
@@ -21,6 +29,7 @@
 // stride uniform across clips).
 #include <cmath>
 #include <cstdlib>
+#include <cstring>
 #include <new>
 #include <vector>
 
@@ -35,12 +44,27 @@ constexpr int kSamples = 480000, kFft = 400, kHop = 160, kFrames = 3000;
 constexpr int kBins = kFft / 2 + 1;               // 201
 constexpr int kFramesPad = kSamples / kHop + 3;   // 3003 frame rows per clip
 constexpr int kClipStride = kFramesPad * kHop;    // 480,480 padded samples per clip
-constexpr int kBasisRows = 404;                   // cos k = 0..200, sin k = 0..200, two zero rows
 constexpr int kPowCols = 204;                     // 201 bins + 3 zero columns
-constexpr int kSlack = 512;                       // read past the last clip by its dropped frame rows
-static_assert((kFramesPad - 1) * kHop + kFft <= kClipStride + kSlack, "slack covers the dropped rows");
+constexpr int kWin = 416;                         // 400-sample window padded to 13 k-blocks of 32
+constexpr int kKb = kWin / 32;                    // 13
+constexpr int kBasisK = 3 * kWin;                 // [hi | lo | hi] parts
+constexpr int kBasisN = 512;                      // 2 x 201 interleaved cos / sin rows, zero padded
+constexpr int kSlack = 4 * kHop;                  // read past the last clip by its dropped frame rows
+static_assert((kFramesPad - 1 + 2) * kHop + kHop <= kClipStride + kSlack, "slack covers the last windows");
+static_assert(kHop % 32 == 0 && kWin <= 3 * kHop, "a window is 13 k-blocks over 3 rows of 160 samples");
 
-__global__ void pad_kernel(const float* __restrict__ audio, float* __restrict__ padded, int B) {
+// a rounded to the nearest tf32 (10 fraction bits, ties to even); low 13 bits zero
+__host__ __device__ inline float round_tf32(float a) {
+  uint32_t u;
+  memcpy(&u, &a, 4);
+  u = (u + 0xFFFu + ((u >> 13) & 1u)) & 0xFFFFE000u;
+  float r;
+  memcpy(&r, &u, 4);
+  return r;
+}
+
+// plane 0: the reflect-padded clips rounded to tf32; plane 1 (plane samples on): the remainders
+__global__ void pad_kernel(const float* __restrict__ audio, float* __restrict__ padded, int B, size_t plane) {
   const size_t total = static_cast<size_t>(B) * kClipStride;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -48,22 +72,10 @@ __global__ void pad_kernel(const float* __restrict__ audio, float* __restrict__ 
     int s = static_cast<int>(i - static_cast<size_t>(b) * kClipStride) - kFft / 2;
     if (s < 0) s = -s;                                    // reflect, edge sample not repeated
     if (s >= kSamples) s = 2 * (kSamples - 1) - s;
-    padded[i] = audio[static_cast<size_t>(b) * kSamples + s];
-  }
-}
-
-__global__ void power_kernel(const float* __restrict__ X, float* __restrict__ P, int rows) {
-  const size_t total = static_cast<size_t>(rows) * kPowCols;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t r = i / kPowCols;
-    const int k = static_cast<int>(i - r * kPowCols);
-    float p = 0.f;
-    if (k < kBins) {
-      const float re = X[r * kBasisRows + k], im = X[r * kBasisRows + kBins + k];
-      p = fmaf(re, re, im * im);
-    }
-    P[i] = p;
+    const float a = audio[static_cast<size_t>(b) * kSamples + s];
+    const float hi = round_tf32(a);
+    padded[i] = hi;
+    padded[plane + i] = a - hi;
   }
 }
 
@@ -117,17 +129,27 @@ __global__ void finish_kernel(const float* __restrict__ L, const unsigned* __res
 }
 
 // ------------------------------------------------------------ host constants
-// Windowed DFT basis: row k = w[n] cos(2 pi k n / 400), row 201 + k = w[n] sin(2 pi k n / 400),
-// w the periodic Hann window; angles reduced exactly ((k n) mod 400) and evaluated in double.
+// Windowed DFT basis [kBasisN, kBasisK]: row 2k = w[n] cos(2 pi k n / 400), row
+// 2k + 1 = w[n] sin(2 pi k n / 400), w the periodic Hann window, angles reduced
+// exactly ((k n) mod 400) and evaluated in double, then rounded to fp32 and split
+// into its tf32 part and remainder: columns [0, 416) hold the tf32 parts,
+// [416, 832) the remainders, [832, 1248) the tf32 parts again (n >= 400 and
+// rows >= 402 are zero).
 std::vector<float> dft_basis() {
-  std::vector<float> basis(static_cast<size_t>(kBasisRows) * kFft, 0.f);
+  std::vector<float> basis(static_cast<size_t>(kBasisN) * kBasisK, 0.f);
   const double two_pi = 6.283185307179586476925286766559;
   for (int k = 0; k < kBins; ++k)
     for (int n = 0; n < kFft; ++n) {
       const double w = 0.5 - 0.5 * std::cos(two_pi * n / kFft);
       const double a = two_pi * static_cast<double>((k * n) % kFft) / kFft;
-      basis[static_cast<size_t>(k) * kFft + n] = static_cast<float>(w * std::cos(a));
-      basis[static_cast<size_t>(kBins + k) * kFft + n] = static_cast<float>(w * std::sin(a));
+      const float v[2] = {static_cast<float>(w * std::cos(a)), static_cast<float>(w * std::sin(a))};
+      for (int q = 0; q < 2; ++q) {
+        float* row = &basis[static_cast<size_t>(2 * k + q) * kBasisK];
+        const float hi = round_tf32(v[q]);
+        row[n] = hi;
+        row[kWin + n] = v[q] - hi;
+        row[2 * kWin + n] = hi;
+      }
     }
   return basis;
 }
@@ -170,9 +192,11 @@ EpiParams store_epi(float* out, int ldo) {
 }  // namespace enc
 
 struct enc_frontend {
-  int n_mels = 0, max_batch = 0, device = 0;
-  float *basis = nullptr, *fb = nullptr, *padded = nullptr, *X = nullptr, *P = nullptr, *M = nullptr;
+  int n_mels = 0, max_batch = 0, device = 0, sm_count = 0;
+  size_t plane = 0;   // samples per plane of the padded buffer (tf32 parts, then remainders)
+  float *basis = nullptr, *fb = nullptr, *padded = nullptr, *P = nullptr, *M = nullptr;
   unsigned* cmax = nullptr;
+  CUtensorMap map_frames, map_basis;   // tf32 operands of the DFT
 };
 
 extern "C" {
@@ -183,8 +207,7 @@ ENC_API void enc_frontend_destroy(enc_frontend* h) {
   const bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
   cudaSetDevice(h->device);
   for (void* p : {static_cast<void*>(h->basis), static_cast<void*>(h->fb), static_cast<void*>(h->padded),
-                  static_cast<void*>(h->X), static_cast<void*>(h->P), static_cast<void*>(h->M),
-                  static_cast<void*>(h->cmax)})
+                  static_cast<void*>(h->P), static_cast<void*>(h->M), static_cast<void*>(h->cmax)})
     if (p) cudaFree(p);
   if (have_prev) cudaSetDevice(prev);
   delete h;
@@ -205,12 +228,13 @@ ENC_API enc_status enc_frontend_create(int32_t n_mels, int32_t max_batch, enc_fr
   h->n_mels = n_mels;
   h->max_batch = max_batch;
   h->device = dev;
+  h->sm_count = prop.multiProcessorCount;
   const size_t rows = static_cast<size_t>(max_batch) * kFramesPad;
-  const size_t padded_n = static_cast<size_t>(max_batch) * kClipStride + kSlack;
-  bool ok = cudaMalloc(&h->basis, sizeof(float) * kBasisRows * kFft) == cudaSuccess &&
+  h->plane = static_cast<size_t>(max_batch) * kClipStride + kSlack;
+  const size_t padded_n = 2 * h->plane;
+  bool ok = cudaMalloc(&h->basis, sizeof(float) * kBasisN * kBasisK) == cudaSuccess &&
             cudaMalloc(&h->fb, sizeof(float) * n_mels * kPowCols) == cudaSuccess &&
             cudaMalloc(&h->padded, sizeof(float) * padded_n) == cudaSuccess &&
-            cudaMalloc(&h->X, sizeof(float) * rows * kBasisRows) == cudaSuccess &&
             cudaMalloc(&h->P, sizeof(float) * rows * kPowCols) == cudaSuccess &&
             cudaMalloc(&h->M, sizeof(float) * rows * n_mels) == cudaSuccess &&
             cudaMalloc(&h->cmax, sizeof(unsigned) * max_batch) == cudaSuccess;
@@ -223,6 +247,9 @@ ENC_API enc_status enc_frontend_create(int32_t n_mels, int32_t max_batch, enc_fr
   ok = cudaMemcpy(h->basis, basis.data(), sizeof(float) * basis.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(h->fb, fb.data(), sizeof(float) * fb.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemset(h->padded, 0, sizeof(float) * padded_n) == cudaSuccess;   // the slack stays zero
+  // frames: rows of 160 samples over both planes; basis: [512, 1248]
+  ok = ok && make_tma_2d_f32(&h->map_frames, h->padded, kHop, padded_n / kHop, kHop * sizeof(float), 128) &&
+       make_tma_2d_f32(&h->map_basis, h->basis, kBasisK, kBasisN, kBasisK * sizeof(float), 128);
   if (!ok) {
     enc_frontend_destroy(h);
     return ENC_ERR_CUDA;
@@ -239,11 +266,18 @@ ENC_API enc_status enc_frontend_log_mel(enc_frontend* h, const float* audio, int
   const int rows = B * kFramesPad, nm = h->n_mels;
   cudaError_t e = cudaSuccess;
   auto ok = [&](cudaError_t r) { if (e == cudaSuccess) e = r; return e == cudaSuccess; };
-  pad_kernel<<<4 * 148, 256, 0, stream>>>(audio, h->padded, B);
+  pad_kernel<<<4 * 148, 256, 0, stream>>>(audio, h->padded, B, h->plane);
   ok(cudaGetLastError());
-  ok(launch_sgemm(h->padded, kHop, h->basis, kFft, rows, kBasisRows, kFft, store_epi(h->X, kBasisRows), stream));
-  power_kernel<<<4 * 148, 256, 0, stream>>>(h->X, h->P, rows);
-  ok(cudaGetLastError());
+  GemmTcParams g = {};
+  g.M = rows;
+  g.N = kBasisN;
+  g.num_kb = 3 * kKb;
+  g.a_mode = A_DFT;
+  g.kb_seg = kKb;
+  g.a_lo_rows = static_cast<int>(h->plane / kHop);
+  g.epi.out = h->P;
+  g.epi.ldo = kPowCols;
+  ok(launch_dft_power_tf32(h->map_frames, h->map_basis, g, h->sm_count, stream));
   ok(launch_sgemm(h->P, kPowCols, h->fb, kPowCols, rows, nm, kPowCols, store_epi(h->M, nm), stream));
   ok(cudaMemsetAsync(h->cmax, 0, sizeof(unsigned) * B, stream));
   log_max_kernel<<<dim3(64, B), 256, 0, stream>>>(h->M, nm, h->cmax);

@@ -55,6 +55,10 @@ __device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, 
   } else if (p.a_mode == A_CONV2) {
     if (kb < 2 * p.kb_seg) { x = kb * BK; y = m0; }
     else { x = (kb - 2 * p.kb_seg) * BK; y = m0 + 1; }
+  } else if (p.a_mode == A_DFT) {
+    const int part = kb / p.kb_seg, w = kb - part * p.kb_seg;
+    x = (w % 5) * 32;
+    y = m0 + w / 5 + (part == 2 ? p.a_lo_rows : 0);
   } else {
     x = kb * BK;
     y = m0;
@@ -228,7 +232,28 @@ enum EpiKind : int {
   EK_GENERIC = 0,   // per-thread stores (conv2 scatter + position table, projector scatter)
   EK_RESID = 1,     // fp32 residual via TMA reduce-add
   EK_STORE = 2,     // bf16 output via TMA store (plain rows, conv1)
+  EK_POWER = 3,     // tf32 operands; out[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2 (log-mel front end)
 };
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 operands read as tf32, fp32 accumulate).
+__device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::tf32: fp32 accumulator, tf32 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int m, int n) {
+  return (1u << 4)                                // D format: f32
+         | (2u << 7)                              // A format: tf32
+         | (2u << 10)                             // B format: tf32
+         | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
+}
 template <int BN, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
@@ -264,13 +289,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
 
+  // producer lane: bit s of `armed` = ring slot s received a load, whose phase parity is bit s of armed_phase
+  uint32_t armed = 0, armed_phase = 0;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      uint32_t armed = 0, armed_phase = 0;   // bit s: slot s holds a load; its phase parity
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -279,9 +305,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
           int ax, ay;
           a_coords(p, m0, kb, ax, ay);
           tma_load_2d(sA + stage * C::kABytes, &map_a, &full[stage], ax, ay);
+          // a k-block is 128 bytes of K: 64 bf16 or 32 tf32 elements
+          constexpr int kx = kEpi == EK_POWER ? 32 : BK;
 #pragma unroll
           for (int half_b = 0; half_b < BN / 128; ++half_b)   // weight maps use 128-row boxes
-            tma_load_2d(sB + stage * C::kBBytes + half_b * (128 * BK * 2), &map_b, &full[stage], kb * BK,
+            tma_load_2d(sB + stage * C::kBBytes + half_b * (128 * BK * 2), &map_b, &full[stage], kb * kx,
                         n0 + half_b * 128);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
@@ -291,15 +319,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       if (!ok) {
         set_status(p.status, kDevTimeout);
         *abort_v = 1;
-        // let copies already in flight land before the CTA's shared memory goes away
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // The whole warp walks the schedule and one elected lane issues and commits.
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+    constexpr bool kTf32 = kEpi == EK_POWER;
+    constexpr uint32_t idesc = kTf32 ? idesc_tf32_f32(BM, BN) : idesc_bf16_f32(BM, BN);
     const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA)), bdesc0 = smem_desc_sw128(smem_u32(sB));
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
@@ -316,9 +342,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(stage) * (C::kBBytes >> 4);
         if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K inside the swizzled row
-            umma_f16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < BK / 16; ++k) {   // +32 bytes along K inside the swizzled row
+            if constexpr (kTf32)
+              umma_tf32_ss(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                           idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_f16_ss(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                          idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit(&empty[stage]);
         }
         __syncwarp();
@@ -360,6 +391,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       } else if constexpr (kEpi == EK_STORE) {
         epi_store_tile<NC / 2>(p.epi, &map_c, m0 + quarter * 32, n0, taddr,
                                reinterpret_cast<uint32_t*>(stage_c + (warp - 2) * 32 * 32), lane);
+      } else if constexpr (kEpi == EK_POWER) {
+        // columns 2k and 2k+1 hold the cos and sin parts of bin k: 16 bins per 32 columns
+        float* prow = reinterpret_cast<float*>(p.epi.out) + (size_t)r * p.epi.ldo;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+          tmem_wait_ld();
+          const int k0 = (n0 + c * 32) >> 1;
+          if (r < p.M && k0 < p.epi.ldo) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              float q[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float re = __uint_as_float(v[2 * (i + j)]), im = __uint_as_float(v[2 * (i + j) + 1]);
+                q[j] = fmaf(re, re, im * im);
+              }
+              if (k0 + i < p.epi.ldo) *reinterpret_cast<float4*>(prow + k0 + i) = make_float4(q[0], q[1], q[2], q[3]);
+            }
+          }
+        }
       } else {
         int dst = 0, pe_row = 0;
         bool zero = false;
@@ -378,13 +431,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    if constexpr (kEpi != EK_GENERIC) {
+    if constexpr (kEpi != EK_GENERIC && kEpi != EK_POWER) {
       if (lane == 0) bulk_wait0();   // the bulk stores / reduces have landed
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_v) {
+    // a CTA that gave up may still have copies in flight (issued, never consumed):
+    // let them land before its shared memory goes away
+    for (int s = 0; s < C::kStages; ++s)
+      if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
@@ -407,6 +466,47 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
 //                       CTA's barrier.
 // ---------------------------------------------------------------------------
 constexpr int kPairStages = 6;
+
+// Work units of the pair kernel: the p.num_tiles tiles of 256 x 256 in row-major
+// tile order, except that the last p.tail tiles are each split into two units
+// of 256 x 128 (their column halves). The launcher sets p.tail so that the last
+// wave of a schedule that would run under half full instead runs twice as many
+// units of half the work. Every output element still comes from one unit, with
+// the same K order, so results do not depend on the split.
+struct PairUnit {
+  int m0, n0, width;   // rows m0 .. m0+255, columns n0 .. n0+width-1 (width 256 or 128)
+};
+__device__ __forceinline__ int pair_units(const GemmTcParams& p) { return p.num_tiles + p.tail; }
+__device__ __forceinline__ PairUnit pair_unit(const GemmTcParams& p, int u) {
+  const int nfull = p.num_tiles - p.tail;
+  if (u < nfull) return {(u / p.tiles_n) * 256, (u % p.tiles_n) * 256, 256};
+  const int h = u - nfull, tile = nfull + (h >> 1);
+  return {(tile / p.tiles_n) * 256, (tile % p.tiles_n) * 256 + (h & 1) * 128, 128};
+}
+
+// Epilogue of one CTA's 128 rows of a unit: each epilogue warp drains its TMEM
+// lane quarter over its half of the unit's columns (NC 32-column chunks).
+template <int kEpi, int NC>
+__device__ __forceinline__ void pair_epilogue(const GemmTcParams& p, const CUtensorMap* map_c, int m0, int n0,
+                                              uint32_t taddr, float* stage, int lane, int quarter) {
+  if constexpr (kEpi == EK_RESID) {
+    epi_residual_tile<NC>(p.epi, map_c, m0 + quarter * 32, n0, taddr, stage, lane);
+  } else if constexpr (kEpi == EK_STORE) {
+    epi_store_tile<NC / 2>(p.epi, map_c, m0 + quarter * 32, n0, taddr, reinterpret_cast<uint32_t*>(stage), lane);
+  } else {
+    const int r = m0 + quarter * 32 + lane;
+    int dst = 0, pe_row = 0;
+    bool zero = false;
+    const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
+#pragma unroll 1
+    for (int c = 0; c < NC; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+      tmem_wait_ld();
+      if (row_ok) epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
+    }
+  }
+}
 constexpr uint32_t kPairABytes = 128 * BK * 2;   // this CTA's 128 rows of A
 constexpr uint32_t kPairBBytes = 128 * BK * 2;   // this CTA's 128 rows of B
 constexpr size_t kPairSmemBytes = 1024 + kPairStages * (size_t)(kPairABytes + kPairBBytes) + 1024 +
@@ -457,16 +557,20 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
 
+  // producer lane: bit s of `armed` = ring slot s received a load, whose phase parity is bit s of armed_phase
+  uint32_t armed = 0, armed_phase = 0;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      uint32_t armed = 0, armed_phase = 0;
-      for (int tile = cluster; ok && tile < p.num_tiles; tile += nclusters) {
-        const int m0 = (tile / p.tiles_n) * 256 + 128 * static_cast<int>(rank);
-        const int n0 = (tile % p.tiles_n) * BN + 128 * static_cast<int>(rank);
+      for (int u = cluster; ok && u < pair_units(p); u += nclusters) {
+        const PairUnit t = pair_unit(p, u);
+        const int m0 = t.m0 + 128 * static_cast<int>(rank);
+        // this CTA's half of the unit's weight rows; a 128-wide unit uses the
+        // first 64 rows of each CTA's 128-row box (the rest is loaded and unused)
+        const int n0 = t.n0 + (t.width / 2) * static_cast<int>(rank);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
@@ -483,22 +587,19 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
       if (!ok) {
         set_status(p.status, kDevTimeout);
         *abort_v = 1;
-        // the first CTA's barriers track the copies; let them land before leaving
-        if (leader)
-          for (int s = 0; s < kPairStages; ++s)
-            if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // first CTA only: the whole warp walks the schedule, one elected lane issues
     if (leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(256, BN), idesc_half = idesc_bf16_f32(256, BN / 2);
       const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA)), bdesc0 = smem_desc_sw128(smem_u32(sB));
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int tile = cluster; ok && tile < p.num_tiles; tile += nclusters) {
+      for (int u = cluster; ok && u < pair_units(p); u += nclusters) {
+        const uint32_t idesc = pair_unit(p, u).width == BN ? idesc_full : idesc_half;
         if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_v, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -539,36 +640,21 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
     const uint32_t tempty_leader[2] = {peer_addr(&tempty[0], 0), peer_addr(&tempty[1], 0)};
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cluster; tile < p.num_tiles; tile += nclusters) {
-      const int m0 = (tile / p.tiles_n) * 256 + 128 * static_cast<int>(rank);
-      const int n0 = (tile % p.tiles_n) * BN + half * (BN / 2);
+    for (int u = cluster; u < pair_units(p); u += nclusters) {
+      const PairUnit t = pair_unit(p, u);
+      const int m0 = t.m0 + 128 * static_cast<int>(rank);
+      const int n0 = t.n0 + half * (t.width / 2);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_v, kWaitLimitNs)) {
         set_status(p.status, kDevTimeout);
         *abort_v = 1;
         break;
       }
       tc_fence_after();
-      const int r = m0 + quarter * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
-      if constexpr (kEpi == EK_RESID) {
-        epi_residual_tile<NC>(p.epi, &map_c, m0 + quarter * 32, n0, taddr, stage_c + (warp - 2) * 32 * 32, lane);
-      } else if constexpr (kEpi == EK_STORE) {
-        epi_store_tile<NC / 2>(p.epi, &map_c, m0 + quarter * 32, n0, taddr,
-                               reinterpret_cast<uint32_t*>(stage_c + (warp - 2) * 32 * 32), lane);
-      } else {
-        int dst = 0, pe_row = 0;
-        bool zero = false;
-        const bool row_ok = (r < p.M) && epi_row(p.epi, r, dst, pe_row, zero);
-#pragma unroll 1
-        for (int c = 0; c < NC; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
-          tmem_wait_ld();
-          if (row_ok)
-            epi_apply_run<bf16, 32>(p.epi, dst, pe_row, zero, n0 + c * 32, reinterpret_cast<const float*>(v));
-        }
-      }
+                             static_cast<uint32_t>(acc * BN + half * (t.width / 2));
+      float* stage = stage_c + (warp - 2) * 32 * 32;
+      if (t.width == BN) pair_epilogue<kEpi, NC>(p, &map_c, m0, n0, taddr, stage, lane, quarter);
+      else pair_epilogue<kEpi, NC / 2>(p, &map_c, m0, n0, taddr, stage, lane, quarter);
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader[acc]);
       acc ^= 1;
@@ -581,6 +667,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
+  if (warp == 0 && lane == 0 && leader && *abort_v) {
+    // the first CTA's stage barriers count both CTAs' copies: after a failure, let
+    // every copy issued into the pair's rings land before either CTA leaves
+    for (int s = 0; s < kPairStages; ++s)
+      if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, nullptr, kWaitLimitNs / 4);
+  }
   cluster_sync();   // no CTA leaves while its pair may still read its memory
   if (warp == 1) {
     tc_fence_after();
@@ -659,6 +751,30 @@ bool make_resid_map(CUtensorMap* map, const float* resid, uint64_t rows, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tma_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
+                     uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn || !base) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (pitch_bytes & 15u)) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_dft_power_tf32(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
+                                  cudaStream_t stream) {
+  if (p.M <= 0) return cudaSuccess;
+  if (p.N % 128 || p.a_mode != A_DFT || !p.epi.out) return cudaErrorInvalidValue;
+  p.tiles_n = p.N / 128;
+  p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
+  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+  return launch_one<128, EK_POWER>(map_a, map_b, map_a, p, grid, stream);
+}
+
 template <int kEpi>
 cudaError_t launch_pair(const CUtensorMap& map_a, const CUtensorMap& map_b, const CUtensorMap& map_c,
                         const GemmTcParams& p, int sm_count, cudaStream_t stream) {
@@ -689,8 +805,14 @@ cudaError_t launch_pair(const CUtensorMap& map_a, const CUtensorMap& map_b, cons
     max_clusters[dev & 63] = n;
     done |= bit;
   }
-  const int clusters = p.num_tiles < max_clusters[dev & 63] ? p.num_tiles : max_clusters[dev & 63];
-  gemm_tc2_kernel<kEpi><<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(map_a, map_b, map_c, p);
+  // a last wave that would run at most half full runs as two 128-wide halves per tile
+  const int ncl = max_clusters[dev & 63];
+  const int tail = p.num_tiles % ncl;
+  GemmTcParams q = p;
+  q.tail = (2 * tail <= ncl) ? tail : 0;
+  const int units = q.num_tiles + q.tail;
+  const int clusters = units < ncl ? units : ncl;
+  gemm_tc2_kernel<kEpi><<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(map_a, map_b, map_c, q);
   return cudaGetLastError();
 }
 

@@ -16,7 +16,11 @@ enc_status validate_config(const enc_config* c);
 void resolve_static_scratch(enc_handle* h);
 
 // ----------------------------------------------------------- tcgen05 GEMM
-enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2 };
+// A_DFT (log-mel front end, tf32): A is read as overlapping windows of 416 fp32
+// samples over rows of 160; k-block kb of a window part (kb / kb_seg: 0 and 1
+// read the rounded-to-tf32 plane, 2 the remainder plane a_lo_rows rows further)
+// is columns (w % 5) * 32 of row m + w / 5, w = kb % kb_seg.
+enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2, A_DFT = 3 };
 
 struct GemmTcParams {
   int M, N;        // output rows / columns (N a multiple of 128)
@@ -26,6 +30,7 @@ struct GemmTcParams {
   int tiles_n;     // filled by the launcher
   int num_tiles;   // filled by the launcher
   int tail;        // SM-pair kernel: the last `tail` tiles run as two 256 x 128 halves (launcher)
+  int a_lo_rows;   // A_DFT: row offset of the remainder plane
   EpiParams epi;
   int* status;
 };
@@ -39,6 +44,18 @@ bool make_out_map(CUtensorMap* map, const void* out, uint64_t rows, uint64_t col
 // 2-D bf16 tensor map with 128-byte swizzle and zero fill outside the tensor.
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
                  uint32_t box_inner, uint32_t box_rows);
+
+// 2-D fp32 tensor map (tf32 operands): 32-element (128-byte) boxes along the
+// inner dimension, 128-byte swizzle, zero fill outside the tensor.
+bool make_tma_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
+                     uint32_t box_rows);
+
+// Windowed DFT and power spectrum on the tensor cores (kind::tf32, 128 x 128
+// tiles on one SM): acc = A W^T over p.num_kb k-blocks of 32 (A_DFT mode),
+// W's rows interleaving the cos and sin basis functions of each bin, so that
+// out[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2 for k < p.epi.ldo (fp32 p.epi.out).
+cudaError_t launch_dft_power_tf32(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
+                                  cudaStream_t stream);
 
 // fp32 [rows, cols] residual matrix as the target of TMA reduce-adds (32 x 32 boxes,
 // 128-byte swizzle). Rows past `rows` are never written.

@@ -8,6 +8,8 @@ and random weights of that architecture.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
     python bench.py --kernel qkv|out|fc1|fc2|attention|frontend|cache [--steps K] [--warmup W]   (one step alone)
+    python bench.py --kernel sidestream [--steps K]   (encoder on a side stream beside a decoder stand-in)
+    python bench.py --kernel block [--steps K]        (the workload's geometry with one encoder block)
 
 One step = one enc_forward over a batch of 16 clips. Multi-GPU (torchrun, one
 process per GPU) runs independent replicas, each with its own batch of 16
@@ -36,6 +38,9 @@ METRIC = "audio-sec/s and TFLOP/s (% of BF16 peak), Whisper-large encoder, B=16,
 UNIT = "audio-s/s"
 FRAMES_PER_SECOND = 100.0          # 16 kHz audio, hop 160
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's published dense BF16 tensor rate of one B200 (its 4.5 PFLOP/s figure
+# assumes 2:4 sparsity); reported beside the measured peaks
+PUBLISHED_DENSE_BF16_TFLOPS = 2250.0
 GEMM_CLASSES = ("conv1", "conv2", "qkv", "out", "fc1", "fc2", "proj1", "proj2")
 
 
@@ -103,39 +108,48 @@ def oracle_sample(cfg, w, mel_clip, length, layers):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(cfg, layers=8):
-    """The oracle on the host cores, on a bounded sample of the same workload."""
+# Both CPU legs (cpu_baseline and --impl reference) time the same sample: one
+# clip of the workload through the conv stem, ORACLE_SAMPLE_BLOCKS of its
+# blocks and the final LayerNorm, converted to audio-s/s at the full workload's
+# FLOPs per audio second.
+ORACLE_SAMPLE_BLOCKS = 4
+
+
+def oracle_sample_setup(cfg):
     lengths = S.make_lengths(cfg)
-    w = S.make_weights(cfg, layers=list(range(layers)))
+    w = S.make_weights(cfg, layers=list(range(ORACLE_SAMPLE_BLOCKS)))
     mel = S.mel_clip(cfg, 0)
-    secs = oracle_sample(cfg, w, mel, lengths[0], layers)
-    sample_flops = workload_flops(cfg, lengths[:1], layers)
+    sample_flops = workload_flops(cfg, lengths[:1], ORACLE_SAMPLE_BLOCKS)
     flops_per_audio_s = workload_flops(cfg, lengths) / (float(np.sum(lengths)) / FRAMES_PER_SECOND)
+    desc = (f"1 clip ({lengths[0]} frames), conv stem + {ORACLE_SAMPLE_BLOCKS} of {cfg.n_layers} blocks + final "
+            f"LN, float64 numpy/BLAS; audio-s/s at the full workload's FLOPs per audio second")
+    return lengths, w, mel, sample_flops, flops_per_audio_s, desc
+
+
+def cpu_baseline(cfg, repeats=5):
+    """The oracle on the host cores, on a bounded sample of the same workload
+    (the median of `repeats` runs of the common sample, about 10 s in all)."""
+    lengths, w, mel, sample_flops, flops_per_audio_s, desc = oracle_sample_setup(cfg)
+    times = [oracle_sample(cfg, w, mel, lengths[0], ORACLE_SAMPLE_BLOCKS) for _ in range(repeats)]
+    secs = statistics.median(times)
     return {"value": sample_flops / secs / flops_per_audio_s, "unit": UNIT, "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": (f"1 clip ({lengths[0]} frames), conv stem + {layers} of {cfg.n_layers} blocks + final LN, "
-                       f"float64 numpy/BLAS, {secs:.2f} s; audio-s/s at the full workload's FLOPs per audio second"),
+            "kind": "oracle", "sample": f"median of {repeats} runs of: {desc}; {secs:.2f} s per run",
             "seconds": secs}
 
 
 def run_reference(args, cfg):
-    """--impl reference: the oracle (float64, host cores) timed on this workload."""
+    """--impl reference: the oracle (float64, host cores) timed on this workload,
+    one run of the common sample per step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    layers = 1
-    lengths = S.make_lengths(cfg)
-    w = S.make_weights(cfg, layers=list(range(layers)))
-    mel = S.mel_clip(cfg, 0)
+    lengths, w, mel, sample_flops, flops_per_audio_s, desc = oracle_sample_setup(cfg)
     for _ in range(args.warmup):
-        oracle_sample(cfg, w, mel, lengths[0], layers)
-    times = [oracle_sample(cfg, w, mel, lengths[0], layers) for _ in range(args.steps)]
+        oracle_sample(cfg, w, mel, lengths[0], ORACLE_SAMPLE_BLOCKS)
+    times = [oracle_sample(cfg, w, mel, lengths[0], ORACLE_SAMPLE_BLOCKS) for _ in range(args.steps)]
     tot = sum(times)
-    sample_flops = workload_flops(cfg, lengths[:1], layers)
-    flops_per_audio_s = workload_flops(cfg, lengths) / (float(np.sum(lengths)) / FRAMES_PER_SECOND)
     value = sample_flops * args.steps / tot / flops_per_audio_s
-    sample = (f"each step: 1 clip ({lengths[0]} frames), conv stem + {layers} of {cfg.n_layers} blocks + final LN, "
-              f"float64 numpy/BLAS; audio-s/s at the full workload's FLOPs per audio second")
+    sample = f"each step: {desc}"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -294,7 +308,23 @@ def run_kernel(args, cfg):
     n = cfg.frames // 2
     M, d, f, H = cfg.batch * n, cfg.d_model, cfg.ffn_dim, cfg.n_heads
     g = torch.Generator(device="cuda").manual_seed(cfg.seed)
-    if args.kernel == "cache":
+    if args.kernel == "block":
+        # every kernel of a forward once (stem, one block with its fused LayerNorms, final LN)
+        from audio_encoder_tower_b200 import Encoder
+        one = cfg.replace(n_layers=1)
+        w_dev = {k: torch.from_numpy(v).to(device="cuda", dtype=torch.bfloat16)
+                 for k, v in S.make_weights(one).items()}
+        enc = Encoder(n_mels=one.n_mels, d_model=one.d_model, n_layers=1, n_heads=one.n_heads,
+                      ffn_dim=one.ffn_dim, max_frames=one.frames, max_batch=one.batch, dtype=one.dtype,
+                      pool_step=one.pool_step, proj_hidden=one.proj_hidden, proj_out=one.proj_out,
+                      attn_chunk=one.attn_chunk, weights=w_dev)
+        del w_dev
+        mel = torch.from_numpy(S.make_mel(one)).to(device="cuda", dtype=torch.bfloat16)
+        lengths = S.make_lengths(one)
+        launch = lambda: enc.forward(mel, lengths)   # noqa: E731
+        flops = workload_flops(one, lengths)
+        shape = {"clips": one.batch, "layers": 1, "audio_s": float(np.sum(lengths)) / FRAMES_PER_SECOND}
+    elif args.kernel == "cache":
         from audio_encoder_tower_b200 import Cache, Encoder
         w_np = S.make_weights(cfg)
         w_dev = {k: torch.from_numpy(v).to(device="cuda", dtype=torch.bfloat16) for k, v in w_np.items()}
@@ -355,9 +385,116 @@ def run_kernel(args, cfg):
     ms = e0.elapsed_time(e1) / args.steps
     line = {"kernel": args.kernel, "workload": cfg.name, "shape": shape, "launches": args.steps,
             "ms_per_launch": ms, "tflops": flops / ms / 1e9}
-    if args.kernel in ("frontend", "cache"):
+    if args.kernel in ("frontend", "cache", "block"):
         line["audio_s_per_s"] = shape["audio_s"] / (ms / 1e3)
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------ encoder side stream
+# A decoder-like stand-in for the side-stream measurement: per layer the four
+# projections of a 3072-wide transformer LLM (the width the Voxtral projector
+# maps into): fused q/k/v 3072 -> 6144, attention output 4096 -> 3072, gate and
+# up 3072 -> 2 x 8192, down 8192 -> 3072, at M = 64 tokens (one decode step of
+# 64 sequences), each a tcgen05 GEMM of this library (enc_linear_bf16).
+DECODER_WIDTH, DECODER_LAYERS, DECODER_TOKENS = 3072, 30, 64
+DECODER_SHAPES = [(6144, 3072), (3072, 4096), (16384, 3072), (3072, 8192)]   # (N, K) per layer
+
+
+def run_sidestream(args, cfg):
+    """The encoder on a low-priority side stream while the decoder stand-in runs
+    decode steps on a high-priority stream ("Multimodal Encoder Side Stream"):
+    each workload alone, then both at once, timed with CUDA events on their own
+    streams. Reports per-forward and per-decode-step times alone and overlapped,
+    and the overlap gain = (sum of the times alone) / (time of both at once)."""
+    import torch
+    from audio_encoder_tower_b200 import Encoder
+    from audio_encoder_tower_b200.binding import linear_bf16
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w_np = S.make_weights(cfg)
+    w_dev = {k: torch.from_numpy(v).to(device=dev, dtype=torch.bfloat16) for k, v in w_np.items()}
+    del w_np
+    enc = Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
+                  ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=cfg.batch, dtype=cfg.dtype,
+                  pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
+                  attn_chunk=cfg.attn_chunk, weights=w_dev)
+    del w_dev
+    lengths = S.make_lengths(cfg)
+    mel = torch.from_numpy(S.make_mel(cfg)).to(device=dev, dtype=torch.bfloat16)
+    _, p_out, d_out = enc.output_positions(cfg.batch, lengths)
+    out = torch.empty((cfg.batch, p_out, d_out), dtype=torch.bfloat16, device=dev)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed)
+    dec_w = [[(torch.randn(n, k, device=dev, generator=g) * 0.02).to(torch.bfloat16) for n, k in DECODER_SHAPES]
+             for _ in range(DECODER_LAYERS)]
+    dec_x = {k: torch.randn(DECODER_TOKENS, k, device=dev, generator=g).to(torch.bfloat16)
+             for k in {k for _, k in DECODER_SHAPES}}
+    dec_y = {n: torch.empty(DECODER_TOKENS, n, device=dev, dtype=torch.bfloat16) for n, _ in DECODER_SHAPES}
+    s_enc = torch.cuda.Stream(dev, priority=0)     # background: the encoder
+    s_dec = torch.cuda.Stream(dev, priority=-1)    # latency-bound: the decoder
+
+    def decode_step():
+        for layer in dec_w:
+            for (n, k), wt in zip(DECODER_SHAPES, layer):
+                linear_bf16(dec_x[k], wt, out=dec_y[n], stream=s_dec)
+
+    def timed(n_enc, n_dec):
+        """n_enc forwards on s_enc and n_dec decode steps on s_dec, started together.
+        Returns (ms of the encoder span, per-step decode ms list, ms of the whole)."""
+        torch.cuda.synchronize(dev)
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(torch.cuda.current_stream(dev))
+        s_enc.wait_event(start)
+        s_dec.wait_event(start)
+        e_end = torch.cuda.Event(enable_timing=True)
+        d_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_dec + 1)]
+        d_ev[0].record(s_dec)
+        i_enc = i_dec = 0
+        while i_enc < n_enc or i_dec < n_dec:   # interleave the host's enqueueing of the two streams
+            if i_enc < n_enc:
+                enc.forward(mel, lengths, out, s_enc)
+                i_enc += 1
+            for _ in range(2):
+                if i_dec < n_dec:
+                    decode_step()
+                    i_dec += 1
+                    d_ev[i_dec].record(s_dec)
+        e_end.record(s_enc)
+        torch.cuda.synchronize(dev)
+        enc_ms = start.elapsed_time(e_end) if n_enc else 0.0
+        dec = [d_ev[i].elapsed_time(d_ev[i + 1]) for i in range(n_dec)]
+        whole = max(enc_ms, start.elapsed_time(d_ev[n_dec]) if n_dec else 0.0)
+        return enc_ms, dec, whole
+
+    for _ in range(max(args.warmup, 3)):
+        enc.forward(mel, lengths, out, s_enc)
+        decode_step()
+    torch.cuda.synchronize(dev)
+    n_enc = max(args.steps, 3)
+    enc_alone, _, _ = timed(n_enc, 0)
+    t_enc = enc_alone / n_enc
+    _, dec_alone, _ = timed(0, 20)
+    t_dec = statistics.median(dec_alone)
+    n_dec = max(1, int(round(enc_alone / t_dec)))   # decode steps spanning the encoder's run
+    enc_both, dec_both, whole = timed(n_enc, n_dec)
+    enc.status(s_enc)
+    enc.close()
+    q = lambda v, f: sorted(v)[min(len(v) - 1, int(f * len(v)))]   # noqa: E731
+    line = {"kernel": "sidestream", "workload": cfg.name,
+            "decoder_stand_in": {"width": DECODER_WIDTH, "layers": DECODER_LAYERS, "tokens": DECODER_TOKENS,
+                                 "gemms_per_layer": [f"{k}->{n}" for n, k in DECODER_SHAPES],
+                                 "kernel": "enc_linear_bf16 (tcgen05 GEMM)", "stream_priority": "high"},
+            "encoder": {"stream_priority": "low", "forwards": n_enc, "ms_alone": t_enc,
+                        "ms_overlapped": enc_both / n_enc, "slowdown": (enc_both / n_enc) / t_enc,
+                        "audio_s_per_s_alone": cfg.batch * cfg.frames / FRAMES_PER_SECOND / (t_enc / 1e3),
+                        "audio_s_per_s_overlapped": cfg.batch * cfg.frames / FRAMES_PER_SECOND /
+                        (enc_both / n_enc / 1e3)},
+            "decoder": {"steps": n_dec, "ms_alone_median": t_dec, "ms_alone_p90": q(dec_alone, 0.9),
+                        "ms_overlapped_median": statistics.median(dec_both), "ms_overlapped_p90": q(dec_both, 0.9),
+                        "slowdown": statistics.median(dec_both) / t_dec},
+            "ms_both_at_once": whole, "ms_sum_alone": n_enc * t_enc + n_dec * t_dec,
+            "overlap_gain": (n_enc * t_enc + n_dec * t_dec) / whole}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 # ---------------------------------------------------------------- our arm
@@ -369,10 +506,13 @@ def main():
     ap.add_argument("--config", default="large_b16", choices=S.CONFIG_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention", "frontend", "cache"],
+    ap.add_argument("--kernel", choices=["qkv", "out", "fc1", "fc2", "attention", "frontend", "cache", "sidestream",
+                                        "block"],
                     help="time one layer kernel of the workload alone (profiling aid)")
     args = ap.parse_args()
     cfg = S.CONFIGS[args.config]
+    if args.kernel == "sidestream":
+        return run_sidestream(args, cfg)
     if args.kernel:
         return run_kernel(args, cfg)
     args.warmup = max(args.warmup, 3)
@@ -532,6 +672,7 @@ def main():
             "tflops": world * tflops,
             "frac_bf16_peak": tflops / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
             "frac_bf16_peak_sustained": tflops / peak_tf,
+            "frac_bf16_published_dense_peak": tflops / PUBLISHED_DENSE_BF16_TFLOPS,
             "peaks": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
             "roofline": roofline,
             "kernels": kernels,

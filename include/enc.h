@@ -63,9 +63,20 @@ typedef enum enc_status {
   ENC_ERR_OOM = 3,           /* device or pinned allocation failed */
   ENC_ERR_CUDA = 4,          /* a CUDA runtime call or a kernel launch failed */
   ENC_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out (status word) */
-  ENC_ERR_DEVICE_CHECK = 6   /* reserved for a device-side range check (status word); the host
-                                validates every input the kernels index by, so no kernel sets it */
+  ENC_ERR_DEVICE_CHECK = 6   /* enc_check_guards: a guard region around a workspace buffer was
+                                written (no kernel sets it in the status word: the host
+                                validates every input the kernels index by) */
 } enc_status;
+
+/*
+ * enc_config.flags: ENC_FLAG_GUARD surrounds every workspace buffer of the
+ * handle (time-major mel, conv1 output, residual stream, LN output, QKV,
+ * attention output, FFN hidden, projector buffers, clip offsets, status word)
+ * with 256 KiB guard regions filled with the byte 0xA5, so
+ * that enc_check_guards can detect a kernel that wrote outside its buffer.
+ * It costs 512 KiB of device memory per buffer and nothing per forward.
+ */
+#define ENC_FLAG_GUARD 1u
 
 typedef enum enc_dtype {
   ENC_DTYPE_BF16 = 0,
@@ -87,7 +98,7 @@ typedef struct enc_config {
   int32_t proj_out;      /* projector output width (multiple of 128) */
   float ln_eps;          /* LayerNorm epsilon (1e-5) */
   int32_t dtype;         /* enc_dtype */
-  uint32_t flags;        /* reserved, must be 0 */
+  uint32_t flags;        /* 0, or ENC_FLAG_GUARD; other bits are reserved and rejected */
   int32_t attn_chunk;    /* 0: full bidirectional attention within each clip; > 0: block-local
                             attention, position i of a clip attending only within its chunk of
                             attn_chunk positions (MiniCPM-o-2.6, "(2) AUDIO": audio_chunk_length
@@ -202,6 +213,28 @@ ENC_API void enc_destroy(enc_handle *h);
 ENC_API const char *enc_status_string(enc_status s);
 
 /* Library-owned device bytes: repacked weights and workspace (for reporting; no passage). */
+
+/*
+ * Guard-band check of a handle created with ENC_FLAG_GUARD (no passage: a
+ * race and overrun detector of this library). Synchronises the device, copies
+ * every guard region to the host and compares it with the fill byte: a plain
+ * device-to-host read, nothing on the device can fault. Returns ENC_OK when
+ * every guard is intact, ENC_ERR_DEVICE_CHECK when one is not (what, if not
+ * NULL, receives a description such as "qkv: byte +4096 past the end of the
+ * buffer changed", truncated to what_len), ENC_ERR_INVALID_ARG for a handle
+ * without guards. The static-scratch forward's workspace has no guards.
+ */
+ENC_API enc_status enc_check_guards(enc_handle *h, char *what, size_t what_len);
+
+/*
+ * Self-test of enc_check_guards without a kernel: changes one byte of a guard
+ * region of workspace buffer `buffer` (allocation order, 0 = time-major mel)
+ * with a host-side cudaMemset (offset < 0: byte -offset before the buffer;
+ * offset > 0: byte offset - 1 past its end, |offset| <= 262144), checks that
+ * enc_check_guards reports that buffer, restores the byte and checks again.
+ * Returns ENC_OK when both checks behaved, ENC_ERR_CUDA when they did not.
+ */
+ENC_API enc_status enc_guard_selftest(enc_handle *h, int32_t buffer, int64_t offset);
 ENC_API size_t enc_device_bytes(const enc_handle *h);
 
 /*

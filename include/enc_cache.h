@@ -11,9 +11,11 @@
  * the other clips of its batch (bit for bit), so a hit returns exactly what a
  * fresh forward would.
  *
- * The key must identify the clip's input: its mel features and its length
- * (for example a content hash computed where the audio arrives); the cache
- * does not read the mel to check it.
+ * The key must identify the clip's input: its mel features and its length.
+ * enc_cache_content_keys derives such a key from the clip's content on the
+ * device; a caller may use its own keys instead (for example a hash computed
+ * where the audio arrives). enc_forward_cached does not read the mel to check
+ * a key: two different clips under one key share one output.
  *
  * Same conventions as enc.h: device pointers, nothing traps, host-detectable
  * errors return before anything is enqueued. All work is enqueued on `stream`;
@@ -33,7 +35,8 @@ typedef struct enc_cache enc_cache;
 /*
  * A cache of `capacity` clip outputs for encoder handle h (which must outlive
  * it), plus staging for h's max_batch clips. Device memory:
- * (capacity + max_batch) output blocks + max_batch mel blocks.
+ * (capacity + max_batch) output blocks + max_batch mel blocks, and 12 bytes per
+ * clip of max_batch for enc_cache_content_keys.
  * Returns ENC_ERR_INVALID_ARG for a null handle or capacity < 1, ENC_ERR_OOM
  * when an allocation fails (nothing is left allocated then).
  */
@@ -49,6 +52,21 @@ ENC_API enc_status enc_cache_create(enc_handle *h, int32_t capacity, enc_cache *
  */
 ENC_API enc_status enc_forward_cached(enc_cache *c, const void *mel, const int32_t *lengths, const uint64_t *keys,
                                       int32_t B, void *out, int32_t *hits, cudaStream_t stream);
+
+/*
+ * Content keys: keys[b] (HOST [B]) is a 64-bit hash of clip b's length and of
+ * its mel values at frames t < lengths[b], the only frames the encoder reads
+ * (frames past the length change neither the output nor the key). Every valid
+ * element contributes the SplitMix64 mix of its position and its bits; the
+ * contributions are summed modulo 2^64 (independent of thread order), and the
+ * sum is mixed with the length's own mix. Two clips with the same length and
+ * the same valid frames get the same key; any other pair collides with a
+ * probability of about 2^-64. The hash kernel is enqueued on `stream`, which
+ * the call then waits for (the keys are host values). mel, lengths, B as for
+ * enc_forward; reads about one byte of HBM per mel byte.
+ */
+ENC_API enc_status enc_cache_content_keys(enc_cache *c, const void *mel, const int32_t *lengths, int32_t B,
+                                          uint64_t *keys, cudaStream_t stream);
 
 /* Number of cached clips (host bookkeeping; no device access). */
 ENC_API int32_t enc_cache_size(const enc_cache *c);

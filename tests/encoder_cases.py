@@ -25,12 +25,14 @@ def to_device(cfg, arrays: dict) -> dict:
     return {k: torch.from_numpy(np.ascontiguousarray(v)).to(device="cuda", dtype=dt) for k, v in arrays.items()}
 
 
-def make_encoder(cfg, dev_w, max_batch=None):
+def make_encoder(cfg, dev_w, max_batch=None, guard=True):
+    """An encoder handle for a test; by default with guard regions around every
+    workspace buffer (ENC_FLAG_GUARD), which run_gpu checks after each forward."""
     from audio_encoder_tower_b200 import Encoder
     return Encoder(n_mels=cfg.n_mels, d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
                    ffn_dim=cfg.ffn_dim, max_frames=cfg.frames, max_batch=max_batch or cfg.batch, dtype=cfg.dtype,
                    pool_step=cfg.pool_step, proj_hidden=cfg.proj_hidden, proj_out=cfg.proj_out,
-                   ln_eps=cfg.ln_eps, attn_chunk=cfg.attn_chunk, weights=dev_w)
+                   ln_eps=cfg.ln_eps, attn_chunk=cfg.attn_chunk, guard=guard, weights=dev_w)
 
 
 def run_gpu(enc, cfg, mel_np, lengths):
@@ -38,6 +40,8 @@ def run_gpu(enc, cfg, mel_np, lengths):
     mel = torch.from_numpy(np.ascontiguousarray(mel_np)).to(device="cuda", dtype=torch_dtype(cfg))
     out = enc.forward(mel, lengths)
     enc.status()
+    if enc.cfg.flags:
+        enc.check_guards()          # no kernel wrote outside its workspace buffer
     return out.float().cpu().numpy().astype(np.float64)
 
 

@@ -70,3 +70,42 @@ def test_argument_errors():
         Cache(enc, 0)
     cache.close()
     enc.close()
+
+
+def test_content_keys():
+    """enc_cache_content_keys: equal clips (same length, same valid frames) get
+    equal keys and hit; one changed valid frame changes the key (a miss); frames
+    past the length change neither the key nor the output; a cached output matches
+    the CPU oracle within the bf16 tolerance."""
+    import torch
+    from tests.encoder_cases import assert_parity, compare, oracle_clip
+    cfg, enc, mel, cache = _setup(8)
+    w = S.make_weights(cfg)
+    mel_np = S.make_mel(cfg.replace(batch=6))
+    lengths = np.array([300, 201, 77, 201], np.int32)
+    sel = mel[[0, 1, 2, 1]].contiguous()
+    keys = cache.content_keys(sel, lengths)
+    assert keys[1] == keys[3] and len(set(keys[:3].tolist())) == 3
+    past = sel.clone()
+    past[1, :, 201:] = 5.0                          # frames past clip 1's length
+    assert np.array_equal(cache.content_keys(past, lengths), keys)
+    assert cache.content_keys(sel, [300, 200, 77, 201])[1] != keys[1]      # the length enters the key
+    one = sel.clone()
+    one[2, 40, 13] = one[2, 40, 13] + 0.5           # one valid frame of clip 2
+    k2 = cache.content_keys(one, lengths)
+    assert k2[2] != keys[2] and np.array_equal(k2[[0, 1, 3]], keys[[0, 1, 3]])
+    out, hits = cache.forward(sel, None, lengths)   # keys from content: clip 3 repeats clip 1
+    assert list(hits) == [0, 0, 0, 0] and cache.size() == 3
+    out2, hits2 = cache.forward(past, None, lengths)
+    assert list(hits2) == [1, 1, 1, 1]
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    _, hits3 = cache.forward(one, None, lengths)
+    assert list(hits3) == [1, 1, 0, 1]
+    got = out2.float().cpu().numpy().astype(np.float64)
+    for b, src in ((1, 1), (2, 2)):
+        n = (int(lengths[b]) + 1) // 2
+        assert_parity(cfg, compare(cfg, got[b], oracle_clip(cfg, w, mel_np[src], lengths[b]), n))
+    enc.status()
+    cache.close()
+    enc.close()

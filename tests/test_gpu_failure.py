@@ -77,3 +77,23 @@ def test_allocation_failure_at_every_point_frees_everything(monkeypatch):
     assert abs(torch.cuda.mem_get_info()[0] - free0) < (8 << 20)
     enc = make_encoder(cfg, w)
     enc.close()
+
+
+def test_guard_regions_report_a_changed_byte():
+    """ENC_FLAG_GUARD: a forward leaves every guard region intact, and a guard
+    byte changed from the host (no kernel, no fault) on either side of a buffer
+    is reported with the buffer's name, then the restored guard passes again."""
+    cfg = S.EncoderConfig(name="guard", n_mels=80, d_model=256, n_layers=1, n_heads=4, ffn_dim=512, frames=200,
+                          batch=2, dtype="bf16", seed=15)
+    enc = make_encoder(cfg, to_device(cfg, S.make_weights(cfg)), guard=True)
+    run_gpu(enc, cfg, S.make_mel(cfg), np.array([200, 77], np.int32))    # checks the guards
+    for buffer, offset in [(0, -1), (0, 1), (2, -262144), (2, 262144), (4, 17), (4, -4096)]:
+        enc.guard_selftest(buffer, offset)
+    enc.check_guards()
+    with pytest.raises(EncError):
+        enc.guard_selftest(0, 0)                # offset 0 is inside the buffer
+    enc.close()
+    plain = make_encoder(cfg, to_device(cfg, S.make_weights(cfg)), guard=False)
+    with pytest.raises(EncError):
+        plain.check_guards()                    # no guards on this handle
+    plain.close()

@@ -79,3 +79,33 @@ def test_attention_bf16(lengths, heads, qscale):
         # bf16 probabilities and bf16 output: a few 2^-8 of the value range
         assert err.max() < 3e-2, (b, float(err.max()))
         assert np.linalg.norm(got[s] - ref) / np.linalg.norm(ref) < 1e-2
+
+
+def test_attention_bf16_many_short_segments():
+    """Segments of at most 192 positions (block-local attention) run as runs of
+    work items per CTA (two CTAs per SM, each looping over its items): 700
+    segments of 1 .. 190 positions x 2 heads is far more items than resident CTAs,
+    so every CTA crosses item boundaries with odd and even tile counts, skipped
+    query tiles and both score buffers. Every segment is compared with the oracle."""
+    import torch
+    from audio_encoder_tower_b200.binding import attention_bf16
+    rng = np.random.default_rng(77)
+    heads = 2
+    d = 64 * heads
+    lengths = rng.integers(1, 191, size=700).tolist()
+    R = sum(lengths)
+    q = _bf16(rng.standard_normal((R, d)))
+    k = _bf16(rng.standard_normal((R, d)))
+    v = _bf16(rng.standard_normal((R, d)))
+    qkv = np.concatenate([q, k, v], axis=1)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    out = attention_bf16(_dev(qkv), _dev(cu, torch.int32), max(lengths), heads)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    worst = 0.0
+    for b, n in enumerate(lengths):
+        s = slice(cu[b], cu[b + 1])
+        ref = O.attention(q[s], k[s], v[s], heads, n)
+        worst = max(worst, float(np.abs(got[s] - ref).max()))
+        assert np.linalg.norm(got[s] - ref) / np.linalg.norm(ref) < 1e-2, b
+    assert worst < 3e-2, worst
