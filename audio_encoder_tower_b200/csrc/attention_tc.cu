@@ -136,17 +136,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr) {
 // lane), written as bf16 pairs over the row's first 48 columns, 32 keys at a
 // time; row sums into ps. kMasked zeroes keys >= kvalid (the clip's last key
 // tile only, so full tiles carry no compare-and-select per key).
-template <bool kMasked>
-__device__ __forceinline__ void softmax_exps(const uint32_t (&v)[kKT], uint32_t tS, float scale_log2, float neg_m,
-                                             int kvalid, float (&ps)[8]) {
-#pragma unroll
-  for (int c = 0; c < kKT / 32; ++c) {
+template <bool kMasked, int c>
+__device__ __forceinline__ void softmax_exps_group(const uint32_t (&v)[kKT], uint32_t tS, float scale_log2,
+                                                   float neg_m, int kvalid, float (&ps)[8]) {
+  {
     uint32_t pk[16];
     if (kMasked && 32 * c >= kvalid) {   // 32 keys past the clip: P = 0 without exponentials
 #pragma unroll
       for (int e = 0; e < 16; ++e) pk[e] = 0u;
       tmem_st_32x32b_x16(tS + static_cast<uint32_t>(16 * c), pk);
-      continue;
+      return;
     }
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
@@ -171,15 +170,22 @@ __device__ __forceinline__ void softmax_exps(const uint32_t (&v)[kKT], uint32_t 
   }
 }
 
+template <bool kMasked>
+__device__ __forceinline__ void softmax_exps(const uint32_t (&v)[kKT], uint32_t tS, float scale_log2, float neg_m,
+                                             int kvalid, float (&ps)[8]) {
+  softmax_exps_group<kMasked, 0>(v, tS, scale_log2, neg_m, kvalid, ps);
+  softmax_exps_group<kMasked, 1>(v, tS, scale_log2, neg_m, kvalid, ps);
+  softmax_exps_group<kMasked, 2>(v, tS, scale_log2, neg_m, kvalid, ps);
+}
+
 }  // namespace
 
 // Work items: (segment b, head h, query tile qt), qt fastest, then h, then b
-// (items of one clip and head are neighbours, so their K/V stay in L2). A CTA
-// takes items blockIdx.x, blockIdx.x + gridDim.x, ...: one item each when the
-// launch has a CTA per item, several when segments are short (block-local
-// attention), so that the next item's Q and K/V loads overlap the current
-// item's work. Items whose query tile starts past the segment are skipped by
-// every role alike.
+// (items of one clip and head run side by side, so their K/V stay in L2). A
+// CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ... (two CTAs per SM),
+// so that its next item's Q and K/V loads and first scores overlap the
+// current item's last tiles and output. Items whose query tile starts past the
+// segment are skipped by every role alike.
 struct AttnItem {
   int start, n, h, q0;
 };
@@ -375,12 +381,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + kColS + static_cast<uint32_t>(bf * kKT);
         uint32_t v[kKT];
-#pragma unroll
-        for (int c = 0; c < kKT / 32; ++c)
+        auto load_group = [&](int c) {
           tmem_ld_32x32b_x32(tS + static_cast<uint32_t>(32 * c), *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
-        tmem_wait_ld();
+        };
         const int kvalid = n - j * kKT;       // keys of this tile inside the segment
         const bool full = kvalid >= kKT;
+#pragma unroll
+        for (int c = 0; c < kKT / 32; ++c) load_group(c);
+        tmem_wait_ld();
         // row maximum of this tile's valid scores, in log2 units
         auto tile_max = [&]() {
           float pm[8];   // eight independent partial maxima, then a tree
@@ -528,10 +536,10 @@ cudaError_t launch_attention_tc(const QkvMaps& maps, bf16* out, const int* cu, i
   const int qtiles = (max_n + kQT - 1) / kQT;
   const long long items = (long long)B * H * qtiles;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  // a CTA per item; segments of one query tile and at most two key tiles (block-local
-  // attention) instead share two CTAs per SM, each taking a run of items
+  // two CTAs per SM, each taking a run of items: a CTA's next Q and K/V loads and
+  // first scores overlap its current item's last tiles and output
   const long long resident = 2LL * sm_count[dev & 63];
-  const int grid = (max_n <= 2 * kKT && items > resident) ? (int)resident : (int)items;
+  const int grid = items > resident ? (int)resident : (int)items;
   attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.kv, out, cu, (int)items, H, qtiles, d,
                                                               0.125f * 1.4426950408889634f, status);
   return cudaGetLastError();

@@ -20,10 +20,13 @@
 //      error-compensated split of the fp32 operands into tf32 pairs. The basis
 //      interleaves cos and sin of each bin, so the epilogue finds both parts of
 //      a bin in adjacent accumulator columns.
-//   4. SGEMM: power x filterbank^T -> mel [B * 3003, n_mels]
-//   5. log_max_kernel: log10(max(mel, 1e-10)) in place over the 3000 frames
+//      The power spectrum is stored split the same way (tf32 part and
+//      remainder planes, 224 bins, zero past 200).
+//   3. tensor cores again: power x filterbank^T -> mel [B * 3003, n_mels] fp32,
+//      the same three-product split over K = 3 x 224.
+//   4. log_max_kernel: log10(max(mel, 1e-10)) in place over the 3000 frames
 //      kept, and the clip's maximum
-//   6. finish_kernel: max(x, clip max - 8), (x + 4) / 4, transposed to
+//   5. finish_kernel: max(x, clip max - 8), (x + 4) / 4, transposed to
 //      [B, n_mels, 3000]
 // Rows 3000..3002 of every clip are computed and dropped (they keep the frame
 // stride uniform across clips).
@@ -44,7 +47,9 @@ constexpr int kSamples = 480000, kFft = 400, kHop = 160, kFrames = 3000;
 constexpr int kBins = kFft / 2 + 1;               // 201
 constexpr int kFramesPad = kSamples / kHop + 3;   // 3003 frame rows per clip
 constexpr int kClipStride = kFramesPad * kHop;    // 480,480 padded samples per clip
-constexpr int kPowCols = 204;                     // 201 bins + 3 zero columns
+constexpr int kPowCols = 224;                     // 201 bins + 23 zero columns: 7 k-blocks of 32
+constexpr int kFbK = 3 * kPowCols;                // [hi | lo | hi] parts of the filterbank
+constexpr int kMelRows = 128;                     // filterbank rows, n_mels zero padded
 constexpr int kWin = 416;                         // 400-sample window padded to 13 k-blocks of 32
 constexpr int kKb = kWin / 32;                    // 13
 constexpr int kBasisK = 3 * kWin;                 // [hi | lo | hi] parts
@@ -162,30 +167,30 @@ double slaney_hz(double mel) {
   return mel < 15.0 ? mel * 200.0 / 3.0 : 1000.0 * std::exp((mel - 15.0) * std::log(6.4) / 27.0);
 }
 
-// [n_mels, kPowCols]: triangles between n_mels + 2 mel-spaced points from 0 Hz to 8 kHz,
-// on bin frequencies k * 40 Hz, each scaled to unit area (2 / (upper - lower edge)).
+// [kMelRows, kFbK]: row m < n_mels holds the triangle between n_mels + 2
+// mel-spaced points from 0 Hz to 8 kHz, on bin frequencies k * 40 Hz, scaled to
+// unit area (2 / (upper - lower edge)), rounded to fp32 and split like the DFT
+// basis: columns [0, 224) its tf32 parts, [224, 448) the remainders, [448, 672)
+// the tf32 parts again; rows >= n_mels and bins > 200 are zero.
 std::vector<float> mel_bank(int n_mels) {
   std::vector<double> edge(n_mels + 2);
   const double top = slaney_mel(8000.0);
   for (int i = 0; i < n_mels + 2; ++i) edge[i] = slaney_hz(top * i / (n_mels + 1));
-  std::vector<float> fb(static_cast<size_t>(n_mels) * kPowCols, 0.f);
+  std::vector<float> fb(static_cast<size_t>(kMelRows) * kFbK, 0.f);
   for (int m = 0; m < n_mels; ++m)
     for (int k = 0; k < kBins; ++k) {
       const double f = 40.0 * k;
       const double rise = (f - edge[m]) / (edge[m + 1] - edge[m]);
       const double fall = (edge[m + 2] - f) / (edge[m + 2] - edge[m + 1]);
       const double t = std::fmax(0.0, std::fmin(rise, fall));
-      fb[static_cast<size_t>(m) * kPowCols + k] = static_cast<float>(t * 2.0 / (edge[m + 2] - edge[m]));
+      const float v = static_cast<float>(t * 2.0 / (edge[m + 2] - edge[m]));
+      float* row = &fb[static_cast<size_t>(m) * kFbK];
+      const float hi = round_tf32(v);
+      row[k] = hi;
+      row[kPowCols + k] = v - hi;
+      row[2 * kPowCols + k] = hi;
     }
   return fb;
-}
-
-EpiParams store_epi(float* out, int ldo) {
-  EpiParams e = {};
-  e.mode = EPI_STORE;
-  e.out = out;
-  e.ldo = ldo;
-  return e;
 }
 
 }  // namespace
@@ -194,9 +199,10 @@ EpiParams store_epi(float* out, int ldo) {
 struct enc_frontend {
   int n_mels = 0, max_batch = 0, device = 0, sm_count = 0;
   size_t plane = 0;   // samples per plane of the padded buffer (tf32 parts, then remainders)
+  int pow_rows = 0;   // rows per plane of the power spectrum (tf32 parts, then remainders)
   float *basis = nullptr, *fb = nullptr, *padded = nullptr, *P = nullptr, *M = nullptr;
   unsigned* cmax = nullptr;
-  CUtensorMap map_frames, map_basis;   // tf32 operands of the DFT
+  CUtensorMap map_frames, map_basis, map_pow, map_fb;   // tf32 operands of the two GEMMs
 };
 
 extern "C" {
@@ -231,11 +237,12 @@ ENC_API enc_status enc_frontend_create(int32_t n_mels, int32_t max_batch, enc_fr
   h->sm_count = prop.multiProcessorCount;
   const size_t rows = static_cast<size_t>(max_batch) * kFramesPad;
   h->plane = static_cast<size_t>(max_batch) * kClipStride + kSlack;
+  h->pow_rows = static_cast<int>(rows);
   const size_t padded_n = 2 * h->plane;
   bool ok = cudaMalloc(&h->basis, sizeof(float) * kBasisN * kBasisK) == cudaSuccess &&
-            cudaMalloc(&h->fb, sizeof(float) * n_mels * kPowCols) == cudaSuccess &&
+            cudaMalloc(&h->fb, sizeof(float) * kMelRows * kFbK) == cudaSuccess &&
             cudaMalloc(&h->padded, sizeof(float) * padded_n) == cudaSuccess &&
-            cudaMalloc(&h->P, sizeof(float) * rows * kPowCols) == cudaSuccess &&
+            cudaMalloc(&h->P, sizeof(float) * 2 * rows * kPowCols) == cudaSuccess &&
             cudaMalloc(&h->M, sizeof(float) * rows * n_mels) == cudaSuccess &&
             cudaMalloc(&h->cmax, sizeof(unsigned) * max_batch) == cudaSuccess;
   if (!ok) {
@@ -249,7 +256,9 @@ ENC_API enc_status enc_frontend_create(int32_t n_mels, int32_t max_batch, enc_fr
        cudaMemset(h->padded, 0, sizeof(float) * padded_n) == cudaSuccess;   // the slack stays zero
   // frames: rows of 160 samples over both planes; basis: [512, 1248]
   ok = ok && make_tma_2d_f32(&h->map_frames, h->padded, kHop, padded_n / kHop, kHop * sizeof(float), 128) &&
-       make_tma_2d_f32(&h->map_basis, h->basis, kBasisK, kBasisN, kBasisK * sizeof(float), 128);
+       make_tma_2d_f32(&h->map_basis, h->basis, kBasisK, kBasisN, kBasisK * sizeof(float), 128) &&
+       make_tma_2d_f32(&h->map_pow, h->P, kPowCols, 2 * rows, kPowCols * sizeof(float), 128) &&
+       make_tma_2d_f32(&h->map_fb, h->fb, kFbK, kMelRows, kFbK * sizeof(float), 128);
   if (!ok) {
     enc_frontend_destroy(h);
     return ENC_ERR_CUDA;
@@ -277,8 +286,18 @@ ENC_API enc_status enc_frontend_log_mel(enc_frontend* h, const float* audio, int
   g.a_lo_rows = static_cast<int>(h->plane / kHop);
   g.epi.out = h->P;
   g.epi.ldo = kPowCols;
+  g.epi.P1 = h->pow_rows;   // the remainder plane of the power spectrum
   ok(launch_dft_power_tf32(h->map_frames, h->map_basis, g, h->sm_count, stream));
-  ok(launch_sgemm(h->P, kPowCols, h->fb, kPowCols, rows, nm, kPowCols, store_epi(h->M, nm), stream));
+  GemmTcParams m = {};
+  m.M = rows;
+  m.N = kMelRows;
+  m.num_kb = 3 * (kPowCols / 32);
+  m.a_mode = A_SPLIT3;
+  m.kb_seg = kPowCols / 32;
+  m.a_lo_rows = h->pow_rows;
+  m.epi.out = h->M;
+  m.epi.ldo = nm;
+  ok(launch_gemm_tf32_f32out(h->map_pow, h->map_fb, m, h->sm_count, stream));
   ok(cudaMemsetAsync(h->cmax, 0, sizeof(unsigned) * B, stream));
   log_max_kernel<<<dim3(64, B), 256, 0, stream>>>(h->M, nm, h->cmax);
   ok(cudaGetLastError());

@@ -59,6 +59,10 @@ __device__ __forceinline__ void a_coords(const GemmTcParams& p, int m0, int kb, 
     const int part = kb / p.kb_seg, w = kb - part * p.kb_seg;
     x = (w % 5) * 32;
     y = m0 + w / 5 + (part == 2 ? p.a_lo_rows : 0);
+  } else if (p.a_mode == A_SPLIT3) {
+    const int part = kb / p.kb_seg;
+    x = (kb - part * p.kb_seg) * 32;
+    y = m0 + (part == 2 ? p.a_lo_rows : 0);
   } else {
     x = kb * BK;
     y = m0;
@@ -232,8 +236,13 @@ enum EpiKind : int {
   EK_GENERIC = 0,   // per-thread stores (conv2 scatter + position table, projector scatter)
   EK_RESID = 1,     // fp32 residual via TMA reduce-add
   EK_STORE = 2,     // bf16 output via TMA store (plain rows, conv1)
-  EK_POWER = 3,     // tf32 operands; out[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2 (log-mel front end)
+  EK_POWER = 3,     // tf32 operands; out[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2, split into tf32 planes
+  EK_F32 = 4,       // tf32 operands; fp32 out[r, n] = acc (log-mel front end: the filterbank)
 };
+// a rounded to the nearest tf32 (10 fraction bits, ties to even); low 13 bits zero
+__device__ __forceinline__ float round_tf32_dev(float a) {
+  return __uint_as_float((__float_as_uint(a) + 0xFFFu + ((__float_as_uint(a) >> 13) & 1u)) & 0xFFFFE000u);
+}
 
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 operands read as tf32, fp32 accumulate).
 __device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -306,7 +315,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
           a_coords(p, m0, kb, ax, ay);
           tma_load_2d(sA + stage * C::kABytes, &map_a, &full[stage], ax, ay);
           // a k-block is 128 bytes of K: 64 bf16 or 32 tf32 elements
-          constexpr int kx = kEpi == EK_POWER ? 32 : BK;
+          constexpr int kx = (kEpi == EK_POWER || kEpi == EK_F32) ? 32 : BK;
 #pragma unroll
           for (int half_b = 0; half_b < BN / 128; ++half_b)   // weight maps use 128-row boxes
             tma_load_2d(sB + stage * C::kBBytes + half_b * (128 * BK * 2), &map_b, &full[stage], kb * kx,
@@ -324,7 +333,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // The whole warp walks the schedule and one elected lane issues and commits.
-    constexpr bool kTf32 = kEpi == EK_POWER;
+    constexpr bool kTf32 = kEpi == EK_POWER || kEpi == EK_F32;
     constexpr uint32_t idesc = kTf32 ? idesc_tf32_f32(BM, BN) : idesc_bf16_f32(BM, BN);
     const uint64_t adesc0 = smem_desc_sw128(smem_u32(sA)), bdesc0 = smem_desc_sw128(smem_u32(sB));
     int stage = 0, acc = 0;
@@ -409,8 +418,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
                 const float re = __uint_as_float(v[2 * (i + j)]), im = __uint_as_float(v[2 * (i + j) + 1]);
                 q[j] = fmaf(re, re, im * im);
               }
-              if (k0 + i < p.epi.ldo) *reinterpret_cast<float4*>(prow + k0 + i) = make_float4(q[0], q[1], q[2], q[3]);
+              if (k0 + i < p.epi.ldo) {
+                float hi[4], lo[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  hi[j] = round_tf32_dev(q[j]);
+                  lo[j] = q[j] - hi[j];
+                }
+                *reinterpret_cast<float4*>(prow + k0 + i) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<float4*>(prow + (size_t)p.epi.P1 * p.epi.ldo + k0 + i) =
+                    make_float4(lo[0], lo[1], lo[2], lo[3]);
+              }
             }
+          }
+        }
+      } else if constexpr (kEpi == EK_F32) {
+        float* orow = reinterpret_cast<float*>(p.epi.out) + (size_t)r * p.epi.ldo;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * 32), v);
+          tmem_wait_ld();
+          const int c0 = n0 + c * 32;
+          if (r < p.M && c0 < p.epi.ldo) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              if (c0 + i < p.epi.ldo)
+                *reinterpret_cast<float4*>(orow + c0 + i) =
+                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                __uint_as_float(v[i + 3]));
           }
         }
       } else {
@@ -431,7 +467,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    if constexpr (kEpi != EK_GENERIC && kEpi != EK_POWER) {
+    if constexpr (kEpi != EK_GENERIC && kEpi != EK_POWER && kEpi != EK_F32) {
       if (lane == 0) bulk_wait0();   // the bulk stores / reduces have landed
     }
   }
@@ -773,6 +809,16 @@ cudaError_t launch_dft_power_tf32(const CUtensorMap& map_a, const CUtensorMap& m
   p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
   const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
   return launch_one<128, EK_POWER>(map_a, map_b, map_a, p, grid, stream);
+}
+
+cudaError_t launch_gemm_tf32_f32out(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p,
+                                    int sm_count, cudaStream_t stream) {
+  if (p.M <= 0) return cudaSuccess;
+  if (p.N % 128 || p.a_mode != A_SPLIT3 || !p.epi.out || p.epi.ldo % 4) return cudaErrorInvalidValue;
+  p.tiles_n = p.N / 128;
+  p.num_tiles = ((p.M + BM - 1) / BM) * p.tiles_n;
+  const int grid = p.num_tiles < sm_count ? p.num_tiles : sm_count;
+  return launch_one<128, EK_F32>(map_a, map_b, map_a, p, grid, stream);
 }
 
 template <int kEpi>

@@ -20,7 +20,10 @@ void resolve_static_scratch(enc_handle* h);
 // samples over rows of 160; k-block kb of a window part (kb / kb_seg: 0 and 1
 // read the rounded-to-tf32 plane, 2 the remainder plane a_lo_rows rows further)
 // is columns (w % 5) * 32 of row m + w / 5, w = kb % kb_seg.
-enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2, A_DFT = 3 };
+// A_SPLIT3 (front end, tf32): k-block kb of part kb / kb_seg is columns
+// (kb % kb_seg) * 32 of row m, in the tf32-part plane for parts 0 and 1 and in
+// the remainder plane a_lo_rows rows further for part 2.
+enum AMode : int { A_PLAIN = 0, A_CONV1 = 1, A_CONV2 = 2, A_DFT = 3, A_SPLIT3 = 4 };
 
 struct GemmTcParams {
   int M, N;        // output rows / columns (N a multiple of 128)
@@ -53,9 +56,15 @@ bool make_tma_2d_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 // Windowed DFT and power spectrum on the tensor cores (kind::tf32, 128 x 128
 // tiles on one SM): acc = A W^T over p.num_kb k-blocks of 32 (A_DFT mode),
 // W's rows interleaving the cos and sin basis functions of each bin, so that
-// out[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2 for k < p.epi.ldo (fp32 p.epi.out).
+// pw[r, k] = acc[r, 2k]^2 + acc[r, 2k+1]^2 for k < p.epi.ldo, stored split as
+// p.epi.out[r, k] = pw rounded to tf32 and, p.epi.P1 rows further, the
+// remainder pw - that (the next tf32 GEMM's operand planes).
 cudaError_t launch_dft_power_tf32(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p, int sm_count,
                                   cudaStream_t stream);
+// fp32 out[r, n] = acc for n < p.epi.ldo (row stride p.epi.ldo), tf32 MMAs, 128 x 128
+// tiles on one SM; A in the A_SPLIT3 mode.
+cudaError_t launch_gemm_tf32_f32out(const CUtensorMap& map_a, const CUtensorMap& map_b, GemmTcParams p,
+                                    int sm_count, cudaStream_t stream);
 
 // fp32 [rows, cols] residual matrix as the target of TMA reduce-adds (32 x 32 boxes,
 // 128-byte swizzle). Rows past `rows` are never written.

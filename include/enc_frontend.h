@@ -17,8 +17,8 @@
  * sin basis on the tensor cores (kind::tf32), with every fp32 operand split
  * into a tf32 part and a tf32 remainder and the three products that matter
  * accumulated in fp32 (about 2^-22 relative to the fp32 product), the power
- * spectrum taken in the same kernel; the filterbank product, log and
- * normalisation run in fp32 on CUDA cores.
+ * spectrum taken in the same kernel. The filterbank product runs the same way
+ * on the tensor cores; log and normalisation run in fp32 on CUDA cores.
  *
  * Same conventions as enc.h: device pointers, row-major, nothing traps;
  * host-detectable errors return before any launch.
@@ -36,7 +36,7 @@ typedef struct enc_frontend enc_frontend;
 
 /*
  * Builds the windowed DFT basis and the filterbank on the current device and
- * allocates the workspace for up to max_batch clips (about 8 MB per clip).
+ * allocates the workspace for up to max_batch clips (about 11 MB per clip).
  * n_mels: 80 or 128. Returns ENC_ERR_INVALID_ARG for other values or
  * max_batch < 1, ENC_ERR_UNSUPPORTED off sm_100, ENC_ERR_OOM / ENC_ERR_CUDA on
  * allocation or copy failure (nothing is left allocated then). *out owns the
