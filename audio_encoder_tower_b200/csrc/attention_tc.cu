@@ -8,19 +8,21 @@
 // Whisper encoder (Qwen2-Audio-7B-Instruct, "(1) AUDIO ENCODER"; head_dim 64,
 // MHA: Voxtral-Mini-3B-2507, "(1) AUDIO ENCODER").
 //
-// One CTA = 128 query rows of one (clip, head); two CTAs share an SM, so one
-// CTA's exponentials overlap the other's waits. K/V stream in tiles of 96 keys.
-//   warp 0      TMA: Q once, then K_j and V_j into a 3-stage ring (128-byte swizzle).
-//   warp 1      MMA issuer (whole warp, one elected lane). S_j = Q K_j^T (M=128, N=96, K=64) goes to score
-//               buffer j%2, so S_{j+1} is ready while the softmax works on S_j.
-//               O += P_j V_j reads P_j from TMEM (A operand in tensor memory):
-//               the softmax writes P_j (bf16) over the first 48 columns of S_j's
-//               own buffer. S_{j+2} reuses that buffer only after P_j V_j has
+// Work items of 128 query rows of one (clip, head); two CTAs share an SM, each
+// taking a run of items, so one CTA's exponentials overlap the other's waits
+// and a CTA's next item's loads overlap its current item. K/V stream in tiles
+// of 96 keys; t below counts a CTA's key tiles across its items.
+//   warp 0      TMA: an item's Q, then K_t and V_t into a 3-stage ring (128-byte swizzle).
+//   warp 1      MMA issuer (whole warp, one elected lane). S_t = Q K_t^T (M=128, N=96, K=64) goes to score
+//               buffer t%2, so S_{t+1} is ready while the softmax works on S_t.
+//               O += P_t V_t reads P_t from TMEM (A operand in tensor memory):
+//               the softmax writes P_t (bf16) over the first 48 columns of S_t's
+//               own buffer. S_{t+2} reuses that buffer only after P_t V_t has
 //               completed.
 //   warps 2, 3  idle (they complete warpgroup 0 for the register split)
 //   warps 4..7  softmax: one query row per thread (its TMEM lane), the whole
 //               96-key score row in registers: exp2, row sum, P. The row's
-//               maximum is taken once, over the first key tile, and kept: later
+//               maximum is taken once, over an item's first key tile, and kept: later
 //               tiles need no max pass. A tile whose row sum exceeds 2^16 (a
 //               score grew far past that maximum) is redone against its own
 //               maximum, with O and l scaled down, after the previous P V has
