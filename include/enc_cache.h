@@ -56,10 +56,12 @@ ENC_API enc_status enc_forward_cached(enc_cache *c, const void *mel, const int32
 /*
  * Content keys: keys[b] (HOST [B]) is a 64-bit hash of clip b's length and of
  * its mel values at frames t < lengths[b], the only frames the encoder reads
- * (frames past the length change neither the output nor the key). Every valid
- * element contributes the SplitMix64 mix of its position and its bits; the
- * contributions are summed modulo 2^64 (independent of thread order), and the
- * sum is mixed with the length's own mix. Two clips with the same length and
+ * (frames past the length change neither the output nor the key). With mix()
+ * the SplitMix64 output finaliser and g = 0x9E3779B97F4A7C15, element (c, t)
+ * of the clip (mel channel c, frame t < lengths[b], T = frames) contributes
+ * mix(((c * T + t) << 32 | its 16- or 32-bit pattern) + g); the contributions
+ * are summed modulo 2^64 (independent of thread order) into s, and
+ * keys[b] = mix(s ^ mix(lengths[b] * g)). Two clips with the same length and
  * the same valid frames get the same key; any other pair collides with a
  * probability of about 2^-64. The hash kernel is enqueued on `stream`, which
  * the call then waits for (the keys are host values). mel, lengths, B as for

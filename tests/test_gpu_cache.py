@@ -109,3 +109,43 @@ def test_content_keys():
     enc.status()
     cache.close()
     enc.close()
+
+
+def _content_key(mel_clip_bits: np.ndarray, length: int, frames: int) -> int:
+    """The documented content key, restated on the host: the sum modulo 2^64 of
+    the SplitMix64 mix of ((c * T + t) << 32 | value bits) + golden over the
+    valid frames t < length, mixed with the mix of length * golden."""
+    mask = (1 << 64) - 1
+    g = 0x9E3779B97F4A7C15
+
+    def mix(z):
+        z &= mask
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & mask
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & mask
+        return z ^ (z >> 31)
+
+    n_mels = mel_clip_bits.shape[0]
+    idx = (np.arange(n_mels, dtype=np.uint64)[:, None] * np.uint64(frames)
+           + np.arange(length, dtype=np.uint64)[None, :])
+    words = (idx << np.uint64(32)) | mel_clip_bits[:, :length].astype(np.uint64)
+    z = (words + np.uint64(g))                        # wraps modulo 2^64
+    z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+    z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+    z = z ^ (z >> np.uint64(31))
+    total = int(np.sum(z, dtype=np.uint64))           # modulo 2^64
+    return mix(total ^ mix(length * g))
+
+
+def test_content_keys_match_their_definition():
+    """The device's content keys equal the documented hash computed on the host,
+    bit for bit, for full and ragged clips."""
+    import torch
+    cfg, enc, mel, cache = _setup(8)
+    lengths = np.array([300, 1, 177, 64], np.int32)
+    sel = mel[:4].contiguous()
+    keys = cache.content_keys(sel, lengths)
+    bits = sel.view(torch.int16).cpu().numpy().view(np.uint16)
+    for b in range(4):
+        assert int(keys[b]) == _content_key(bits[b], int(lengths[b]), cfg.frames), b
+    cache.close()
+    enc.close()
