@@ -67,11 +67,16 @@ __device__ __forceinline__ void store4(OutT* p, float a, float b, float c, float
   }
 }
 
+// One warp per row. Blocks take the rows from the last to the first: the GEMM
+// that updated x before this kernel (out-proj or fc2, tiles in ascending row
+// order) wrote the last rows last, so those are the ones still in L2, and the
+// rows this kernel writes last (the first ones) are those the next GEMM reads
+// first.
 template <typename OutT, int NV>
 __global__ void layernorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                  const float* __restrict__ bta, OutT* __restrict__ y, int rows, float eps) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int row = (gridDim.x - 1 - blockIdx.x) * (blockDim.x >> 5) + warp;
   if (row >= rows) return;
   constexpr int d = NV * 128;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
