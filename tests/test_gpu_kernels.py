@@ -81,6 +81,39 @@ def test_attention_bf16(lengths, heads, qscale):
         assert np.linalg.norm(got[s] - ref) / np.linalg.norm(ref) < 1e-2
 
 
+def test_attention_bf16_late_large_scores():
+    """Scores far above the row maximum taken over a segment's first key tile:
+    every query shares a component u, and keys 250, 1100 and 1400 are 4u, 8u and
+    30u, so their exponentials exceed that maximum's by factors of about 2^41,
+    2^92 and 2^346. Each makes the row's sum for its key tile overflow the bound, so
+    the row moves to a higher maximum and rescales what it has accumulated, the
+    last time by more than 2^126 (the old values drop to zero). Compared with the
+    oracle's softmax, which subtracts the exact maximum."""
+    import torch
+    from audio_encoder_tower_b200.binding import attention_bf16
+    rng = np.random.default_rng(78)
+    heads, lengths = 2, [300, 1500]
+    d = 64 * heads
+    R = sum(lengths)
+    q = rng.standard_normal((R, d)) + 1.0
+    k = rng.standard_normal((R, d))
+    for pos, c in ((250, 4.0), (1100, 8.0), (1400, 30.0)):
+        k[lengths[0] + pos] = c                     # c * u, u = all ones in every head
+    q, k = _bf16(q), _bf16(k)
+    v = _bf16(rng.standard_normal((R, d)))
+    qkv = np.concatenate([q, k, v], axis=1)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    out = attention_bf16(_dev(qkv), _dev(cu, torch.int32), max(lengths), heads)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    for b, n in enumerate(lengths):
+        s = slice(cu[b], cu[b + 1])
+        ref = O.attention(q[s], k[s], v[s], heads, n)
+        assert np.abs(got[s] - ref).max() < 3e-2, b
+        assert np.linalg.norm(got[s] - ref) / np.linalg.norm(ref) < 1e-2, b
+
+
 def test_attention_bf16_many_short_segments():
     """Segments of at most 192 positions (block-local attention) run as runs of
     work items per CTA (two CTAs per SM, each looping over its items): 700
