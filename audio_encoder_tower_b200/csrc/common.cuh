@@ -292,17 +292,34 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// mbar_test with a suspend-time hint: while the phase is incomplete the thread
+// sleeps in the instruction until the phase completes or about `hint_ns` have
+// passed, instead of returning at once to spin (a spinning warp takes issue
+// slots from the warps that share its scheduler).
+__device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete, for at most
 // `limit_ns` nanoseconds or until *abort (when given) becomes non-zero. Returns false when
-// the wait gave up (the caller records the error and unwinds).
+// the wait gave up (the caller records the error and unwinds). Each retry sleeps for at
+// most 20 us, so the limit and the abort flag are looked at every 320 us or sooner.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_test(a, parity)) return true;
-    if ((it & 255u) == 0u) {
+    if (mbar_test_sleep(a, parity, 20000u)) return true;
+    if ((it & 15u) == 0u) {
       if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
