@@ -13,13 +13,19 @@
 // and a CTA's next item's loads overlap its current item. K/V stream in tiles
 // of 96 keys; t below counts a CTA's key tiles across its items.
 //   warp 0      TMA: an item's Q, then K_t and V_t into a 3-stage ring (128-byte swizzle).
-//   warp 1      MMA issuer (whole warp, one elected lane). S_t = Q K_t^T (M=128, N=96, K=64) goes to score
-//               buffer t%2, so S_{t+1} is ready while the softmax works on S_t.
-//               O += P_t V_t reads P_t from TMEM (A operand in tensor memory):
-//               the softmax writes P_t (bf16) over the first 48 columns of S_t's
-//               own buffer. S_{t+2} reuses that buffer only after P_t V_t has
-//               completed.
-//   warps 2, 3  idle (they complete warpgroup 0 for the register split)
+//   warp 1      TMEM allocation; otherwise idle (it completes warpgroup 0 for
+//               the register split).
+//   warp 2      score issuer (whole warp, one elected lane): S_t = Q K_t^T
+//               (M=128, N=96, K=64) goes to score buffer t%2, so S_{t+1} is
+//               ready while the softmax works on S_t. S_{t+2} reuses that buffer
+//               only after P_t V_t has completed.
+//   warp 3      P V issuer (whole warp, one elected lane): O += P_t V_t reads P_t
+//               from TMEM (A operand in tensor memory): the softmax writes P_t
+//               (bf16) over the first 48 columns of S_t's own buffer.
+//               The two issuers sit on two warp schedulers (warp w runs on
+//               scheduler w % 4, beside softmax warp 4 + w % 4): issuing a
+//               tile's ten MMAs from one warp held back the softmax warp that
+//               shares its scheduler, and P V waits for the slowest softmax warp.
 //   warps 4..7  softmax: one query row per thread (its TMEM lane), the whole
 //               96-key score row in registers: exp2, row sum, P. The row's
 //               maximum is taken once, over an item's first key tile, and kept: later
@@ -216,8 +222,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   uint64_t* pv_done = p_full + 2;                 // [2] P_t V_t complete
   uint64_t* o_done = pv_done + 2;                 // every MMA of the i-th item complete: O final
   uint64_t* o_empty = o_done + 1;                 // the softmax has read O of the i-th item
-  uint64_t* drain = o_empty + 1;                  // every MMA of the CTA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = o_empty + 1;                  // [2] every S MMA / every P V MMA of the CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,7 +238,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
     mbar_init(o_done, 1);
     mbar_init(o_empty, 128);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -276,11 +283,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         set_status(status, kDevTimeout);
         *abort_v = 1;
       }
-    } else if (warp == 1) {
+    } else if (warp == 2 || warp == 3) {
       // ------------------------------------------------------------ MMA
-      // The whole warp walks the schedule and one elected lane issues, so the
-      // operands stay warp-uniform (a tcgen05.mma issued from divergent code
-      // costs several times more issue cycles).
+      // Two issuers on two schedulers: warp 2 issues the scores S_t, warp 3 the
+      // products P_t V_t. The whole warp walks the schedule and one elected lane
+      // issues, so the operands stay warp-uniform.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHD) | (1u << 16);   // B (V) MN-major
       constexpr uint64_t kSlotDesc = kKVBytes >> 4;   // one ring slot in descriptor address units
@@ -288,64 +295,71 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sK));
       const uint64_t vdesc0 = smem_desc_sw128_mn(smem_u32(sV));
+      const bool s_role = warp == 2;
       bool issued = false, ok = true;
-      // S_t = Q K_t^T into buffer t % 2, after that buffer's previous P (tile t - 2)
-      // has been read by its P V, and K_t has landed; the last S of an item frees Q
-      auto issue_s = [&](int t, bool last_of_item) {
-        const uint32_t bf = static_cast<uint32_t>(t & 1);
-        if (t >= 2 && !wait_all(&pv_done[bf], static_cast<uint32_t>(((t - 2) >> 1) & 1))) return false;
-        if (!wait_all(&kv_full[slot(t)], fill_parity(t))) return false;
-        tc_fence_after();
-        const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(slot(t)) * kSlotDesc;
-        if (elect_one()) {
-#pragma unroll
-          for (int k = 0; k < kHD / 16; ++k)
-            umma_f16_ss(tmem + kColS + bf * kKT, qdesc + static_cast<uint64_t>(2 * k),
-                        kdesc + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
-          umma_commit(&s_full[bf]);
-          if (last_of_item) umma_commit(q_empty);
-        }
-        __syncwarp();
-        issued = true;
-        return true;
-      };
       int t0 = 0, ic = 0;   // tiles and items of this CTA so far
       for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
         const AttnItem w = attn_item(cu, it, H, qtiles);
         if (w.q0 >= w.n) continue;
         const int nkv = (w.n + kKT - 1) / kKT;
-        ok = wait_all(q_full, static_cast<uint32_t>(ic & 1));
-        for (int j = 0; ok && j < 2 && j < nkv; ++j) ok = issue_s(t0 + j, j == nkv - 1);
-        for (int j = 0; ok && j < nkv; ++j) {
-          const int t = t0 + j;
-          const uint32_t bf = static_cast<uint32_t>(t & 1), use = static_cast<uint32_t>((t >> 1) & 1);
-          ok = wait_all(&p_full[bf], use);
-          // the item's first P V overwrites O: the softmax must have read the previous item's O
-          if (ok && j == 0 && ic > 0) ok = wait_all(o_empty, static_cast<uint32_t>((ic - 1) & 1));
-          if (!ok) break;
-          tc_fence_after();
-          // O += P_t V_t: P_t in the first 48 columns of buffer t % 2, 16 keys (8 columns) per step
-          const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(slot(t)) * kSlotDesc;
-          if (elect_one()) {
+        if (s_role) {
+          ok = wait_all(q_full, static_cast<uint32_t>(ic & 1));
+          // S_t = Q K_t^T into buffer t % 2, after that buffer's previous P (tile t - 2)
+          // has been read by its P V, and K_t has landed; the last S of an item frees Q
+          for (int j = 0; ok && j < nkv; ++j) {
+            const int t = t0 + j;
+            const uint32_t bf = static_cast<uint32_t>(t & 1);
+            if (t >= 2) ok = wait_all(&pv_done[bf], static_cast<uint32_t>(((t - 2) >> 1) & 1));
+            if (ok) ok = wait_all(&kv_full[slot(t)], fill_parity(t));
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(slot(t)) * kSlotDesc;
+            if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < kKT / 16; ++k)
-              umma_f16_ts(tmem + kColO, tmem + kColS + bf * kKT + static_cast<uint32_t>(8 * k),
-                          vdesc + static_cast<uint64_t>(128 * k), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
-            umma_commit(&pv_done[bf]);
-            umma_commit(&kv_empty[slot(t)]);
-            if (j == nkv - 1) umma_commit(o_done);
+              for (int k = 0; k < kHD / 16; ++k)
+                umma_f16_ss(tmem + kColS + bf * kKT, qdesc + static_cast<uint64_t>(2 * k),
+                            kdesc + static_cast<uint64_t>(2 * k), idesc_s, k > 0 ? 1u : 0u);
+              umma_commit(&s_full[bf]);
+              if (j == nkv - 1) umma_commit(q_empty);
+            }
+            __syncwarp();
+            issued = true;
           }
-          __syncwarp();
-          if (j + 2 < nkv) ok = issue_s(t + 2, j + 2 == nkv - 1);
+        } else {
+          for (int j = 0; ok && j < nkv; ++j) {
+            const int t = t0 + j;
+            const uint32_t bf = static_cast<uint32_t>(t & 1), use = static_cast<uint32_t>((t >> 1) & 1);
+            // the softmax has read S_t (so S_t is complete) and written P_t
+            ok = wait_all(&p_full[bf], use);
+            // the item's first P V overwrites O: the softmax must have read the previous item's O
+            if (ok && j == 0 && ic > 0) ok = wait_all(o_empty, static_cast<uint32_t>((ic - 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            // O += P_t V_t: P_t in the first 48 columns of buffer t % 2, 16 keys (8 columns) per step
+            const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(slot(t)) * kSlotDesc;
+            if (elect_one()) {
+#pragma unroll
+              for (int k = 0; k < kKT / 16; ++k)
+                umma_f16_ts(tmem + kColO, tmem + kColS + bf * kKT + static_cast<uint32_t>(8 * k),
+                            vdesc + static_cast<uint64_t>(128 * k), idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+              // K_t was read by S_t, complete before the softmax saw it; V_t by these MMAs
+              umma_commit(&pv_done[bf]);
+              umma_commit(&kv_empty[slot(t)]);
+              if (j == nkv - 1) umma_commit(o_done);
+            }
+            __syncwarp();
+            issued = true;
+          }
         }
         t0 += nkv;
         ++ic;
       }
       if (!ok && lane == 0) { set_status(status, kDevTimeout); *abort_v = 1; }
-      if (issued) {   // every MMA done before TMEM is released: this wait ignores the abort flag
-        if (elect_one()) umma_commit(drain);
+      if (issued) {   // this warp's MMAs done before TMEM is released: this wait ignores the abort flag
+        uint64_t* dr = &drain[s_role ? 0 : 1];
+        if (elect_one()) umma_commit(dr);
         __syncwarp();
-        mbar_wait_warp(drain, 0, nullptr, kWaitNs);
+        mbar_wait_warp(dr, 0, nullptr, kWaitNs);
       }
     }
   } else {
