@@ -532,23 +532,30 @@ bool make_qkv_maps(QkvMaps* maps, const void* qkv, int rows, int d) {
 cudaError_t launch_attention_tc(const QkvMaps& maps, bf16* out, const int* cu, int B, int max_n, int d, int H,
                                 int* status, cudaStream_t stream) {
   if (B <= 0 || max_n <= 0) return cudaSuccess;
-  static unsigned long long done = 0;
-  static int sm_count[64] = {};
+  static DeviceOnce once;
+  static int sm_count[64] = {};   // written under once's mutex, read after its acquire
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
-  if (!(done & (1ull << (dev & 63)))) {
+  cudaError_t setup_error = cudaSuccess;
+  const bool ready = once.run(dev, [&] {
     // setmaxnreg redistributes the registers the CTA was launched with: refuse to
     // launch unless the compiled kernel holds exactly the planned count per thread
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, attention_tc_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sm_count[dev & 63], cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    done |= 1ull << (dev & 63);
-  }
+    if (e == cudaSuccess && fa.numRegs != kRegsLaunch) e = cudaErrorInvalidConfiguration;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    int n = 0;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && n < 1) e = cudaErrorInvalidValue;
+    if (e != cudaSuccess) {
+      setup_error = e;
+      return false;
+    }
+    sm_count[dev & 63] = n;
+    return true;
+  });
+  if (!ready) return setup_error != cudaSuccess ? setup_error : cudaErrorInvalidValue;
   const int qtiles = (max_n + kQT - 1) / kQT;
   const long long items = (long long)B * H * qtiles;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;

@@ -718,30 +718,28 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once, by whichever thread comes first (a function-local static
+  // is initialised exactly once even when threads race for it)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
 template <int BN, int kEpi>
 bool configure_once() {
-  static unsigned long long done = 0;   // bit per device ordinal
+  static DeviceOnce once;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(done & bit)) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)TcCfg<BN>::kSmemBytes) != cudaSuccess)
-      return false;
-    done |= bit;
-  }
-  return true;
+  return once.run(dev, [] {
+    return cudaFuncSetAttribute(gemm_tc_kernel<BN, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)TcCfg<BN>::kSmemBytes) == cudaSuccess;
+  });
 }
 
 template <int BN, int kEpi>
@@ -824,15 +822,18 @@ cudaError_t launch_gemm_tf32_f32out(const CUtensorMap& map_a, const CUtensorMap&
 template <int kEpi>
 cudaError_t launch_pair(const CUtensorMap& map_a, const CUtensorMap& map_b, const CUtensorMap& map_c,
                         const GemmTcParams& p, int sm_count, cudaStream_t stream) {
-  static unsigned long long done = 0;
-  static int max_clusters[64] = {};
+  static DeviceOnce once;
+  static int max_clusters[64] = {};   // written under once's mutex, read after its acquire
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(done & bit)) {
+  cudaError_t setup_error = cudaSuccess;
+  const bool ready = once.run(dev, [&] {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kPairSmemBytes);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      setup_error = e;
+      return false;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sm_count / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -848,9 +849,14 @@ cudaError_t launch_pair(const CUtensorMap& map_a, const CUtensorMap& map_b, cons
     e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<kEpi>, &cfg);
     if (e != cudaSuccess || n < 1) n = sm_count / 2;   // every SM pairs up
     cudaGetLastError();
+    if (n < 1) {
+      setup_error = cudaErrorInvalidValue;
+      return false;
+    }
     max_clusters[dev & 63] = n;
-    done |= bit;
-  }
+    return true;
+  });
+  if (!ready) return setup_error != cudaSuccess ? setup_error : cudaErrorInvalidValue;
   // a last wave that would run at most half full runs as two 128-wide halves per tile
   const int ncl = max_clusters[dev & 63];
   const int tail = p.num_tiles % ncl;

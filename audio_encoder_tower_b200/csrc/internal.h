@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "../../include/enc.h"
 
@@ -12,6 +15,27 @@ namespace enc {
 
 // Geometry checks of enc_create, without the device check (host only).
 enc_status validate_config(const enc_config* c);
+
+// Per-device one-time set-up of a launcher (kernel attributes, occupancy
+// queries), safe when several host threads launch at once: init() runs at most
+// once per device ordinal at a time, under the mutex, and a thread that sees the
+// device's bit set (acquire) also sees everything init() wrote before the bit
+// was published (release). Device ordinals are taken modulo 64. A failed init()
+// leaves the bit clear, so the next call tries again.
+struct DeviceOnce {
+  std::atomic<unsigned long long> done{0};
+  std::mutex m;
+  template <typename F>
+  bool run(int dev, F&& init) {
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    std::lock_guard<std::mutex> lock(m);
+    if (done.load(std::memory_order_relaxed) & bit) return true;
+    if (!init()) return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+  }
+};
 // enc_forward_static_scratch set-up (enc_create): the static workspace's device address.
 void resolve_static_scratch(enc_handle* h);
 
