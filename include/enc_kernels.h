@@ -37,7 +37,9 @@ ENC_API enc_status enc_linear_bf16(const void *A, const void *W, const float *bi
  *        every row must hold finite values (rows of neighbouring clips are
  *        read by a clip's last key tile and masked out)
  *   cu   device int32 [B+1]: clip b owns rows cu[b] .. cu[b+1]-1 (its keys);
- *        cu[B] <= rows
+ *        0 <= cu[0] <= cu[1] <= ... <= cu[B] <= rows. These are device values
+ *        and are not checked: offsets outside this rule make the kernel write
+ *        outside out.
  *   out  bf16 [rows, d] = concat_h softmax(q_h k_h^T / 8) v_h on rows < cu[B]
  * max_n >= max_b (cu[b+1] - cu[b]) (host value). d = 64 * n_heads.
  * status: device int (may be NULL) set to ENC_ERR_TIMEOUT if a bounded wait

@@ -68,6 +68,17 @@ def test_argument_errors():
         cache.forward(mel[:1].contiguous(), keys=[1], lengths=[301])       # length > T
     with pytest.raises(EncError):
         Cache(enc, 0)
+    # B = 0 with valid pointers
+    import ctypes
+    import torch
+    _, p_out, d_out = enc.output_positions(1)
+    out = mel.new_zeros((1, p_out, d_out))
+    keys = np.zeros(1, np.uint64)
+    kp = keys.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64))
+    stream = torch.cuda.current_stream().cuda_stream
+    assert cache.lib.enc_forward_cached(cache.h, mel.data_ptr(), None, kp, 0, out.data_ptr(), None, stream) == 1
+    assert cache.lib.enc_cache_content_keys(cache.h, mel.data_ptr(), None, 0, kp, stream) == 1
+    assert cache.size() == 0
     cache.close()
     enc.close()
 

@@ -50,6 +50,11 @@ def test_silence_and_argument_errors():
     assert torch.all(out == -1.5)                       # log10(1e-10) = -10 -> (-10 + 4) / 4
     with pytest.raises(EncError):
         fe.log_mel(torch.zeros((3, 480000), dtype=torch.float32, device="cuda"))   # B > max_batch
+    out = torch.full((1, 80, 3000), 3.0, dtype=torch.bfloat16, device="cuda")   # B = 0, valid pointers
+    assert fe.lib.enc_frontend_log_mel(fe.h, z.data_ptr(), 0, out.data_ptr(), 0,
+                                       torch.cuda.current_stream().cuda_stream) == 1
+    torch.cuda.synchronize()
+    assert torch.all(out == 3.0)
     fe.close()
     with pytest.raises(EncError):
         Frontend(n_mels=64)

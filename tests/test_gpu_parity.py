@@ -119,6 +119,18 @@ def test_argument_errors():
     big = torch.zeros((cfg.batch + 1, cfg.n_mels, cfg.frames), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(EncError):
         enc.forward(big)
+    # an empty batch (B = 0, valid pointers) is an argument error, reported before
+    # anything is enqueued
+    _, p_out, d_out = enc.output_positions(1)
+    sentinel = torch.full((1, p_out, d_out), 3.0, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for fn in (enc.lib.enc_forward, enc.lib.enc_forward_static_scratch):
+        assert fn(enc.handle, mel.data_ptr(), None, 0, sentinel.data_ptr(), stream) == 1
+    with pytest.raises(EncError) as ei:
+        enc.output_positions(0)
+    assert ei.value.code == 1
+    torch.cuda.synchronize()
+    assert torch.all(sentinel == 3.0)
     enc.status()
     enc.close()
     for kw, code in [(dict(n_heads=3), 2), (dict(d_model=200, n_heads=4), 2), (dict(pool_step=3), 2),
